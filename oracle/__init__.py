@@ -1,0 +1,149 @@
+"""fp64 CPU oracle of the LatentMoE layer forward -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. It shares no code with the CUDA
+library (``latentmoe_layer_b200``); the only common dependency is the seeded
+input generator in ``synth``. The arithmetic lives in ``oracle.c`` (plain
+loops, fp64, OpenMP over tokens); this module only marshals arguments.
+
+What each function computes and which passage it follows is stated in
+``oracle.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+class LmoCfg(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int), ("L", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int),
+                ("G", ctypes.c_int), ("Gk", ctypes.c_int), ("I", ctypes.c_int), ("Is", ctypes.c_int),
+                ("s", ctypes.c_double), ("x_f32", ctypes.c_int), ("fp32_mode", ctypes.c_int)]
+
+
+class LmoWeights(ctypes.Structure):
+    _fields_ = [("router_w", ctypes.c_void_p), ("e_bias", ctypes.c_void_p), ("fc1_w", ctypes.c_void_p),
+                ("fc2_w", ctypes.c_void_p), ("up_w", ctypes.c_void_p), ("down_w", ctypes.c_void_p),
+                ("shared_up_w", ctypes.c_void_p), ("shared_down_w", ctypes.c_void_p)]
+
+
+def build(force: bool = False):
+    srcs = [os.path.join(_HERE, "oracle.c"), os.path.join(_HERE, "oracle.h")]
+    if not force and os.path.exists(_SO) and all(os.path.getmtime(s) <= os.path.getmtime(_SO) for s in srcs):
+        return
+    cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-std=c11", srcs[0], "-o", _SO, "-lm"]
+    r = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+    if r.returncode != 0:
+        raise RuntimeError("oracle build failed:\n" + r.stdout)
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_SO)
+        vp, i64 = ctypes.c_void_p, ctypes.c_int64
+        lib.lmo_round_bf16.argtypes = [ctypes.c_double]
+        lib.lmo_round_bf16.restype = ctypes.c_double
+        lib.lmo_select.argtypes = [vp, vp, vp]
+        lib.lmo_logits.argtypes = [vp, vp, vp, i64, vp]
+        lib.lmo_route.argtypes = [vp, vp, vp, vp, i64, vp, vp]
+        lib.lmo_forward.argtypes = [vp, vp, vp, i64, vp, vp, vp]
+        for f in (lib.lmo_select, lib.lmo_logits, lib.lmo_route, lib.lmo_forward):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def make_cfg(shape, fp32_mode=False, x_f32=None) -> LmoCfg:
+    """shape: any object with H, L, E, k, G, Gk, I, Is, s (and x_f32)."""
+    xf = shape.x_f32 if x_f32 is None else x_f32
+    return LmoCfg(shape.H, shape.L, shape.E, shape.k, shape.G, shape.Gk, shape.I, shape.Is, float(shape.s),
+                  int(bool(xf)), int(bool(fp32_mode)))
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+def _xarr(cfg: LmoCfg, x):
+    return _c(x, np.float32 if cfg.x_f32 else np.uint16)
+
+
+def round_bf16(v: float) -> float:
+    return _get().lmo_round_bf16(float(v))
+
+
+def select(cfg: LmoCfg, c) -> np.ndarray:
+    c = _c(np.asarray(c, dtype=np.float64), np.float64)
+    sel = np.zeros(cfg.k, dtype=np.int32)
+    rc = _get().lmo_select(ctypes.byref(cfg), c.ctypes.data, sel.ctypes.data)
+    if rc != 0:
+        raise ValueError("invalid selection configuration")
+    return sel
+
+
+def logits(cfg: LmoCfg, x, router_w) -> np.ndarray:
+    x = _xarr(cfg, x)
+    rw = _c(router_w, np.uint16)
+    n = x.shape[0]
+    out = np.zeros((n, cfg.E), dtype=np.float64)
+    _get().lmo_logits(ctypes.byref(cfg), x.ctypes.data, rw.ctypes.data, n, out.ctypes.data)
+    return out
+
+
+def route(cfg: LmoCfg, x, router_w, e_bias):
+    x = _xarr(cfg, x)
+    rw = _c(router_w, np.uint16)
+    b = _c(e_bias, np.float32)
+    n = x.shape[0]
+    idx = np.zeros((n, cfg.k), dtype=np.int32)
+    w = np.zeros((n, cfg.k), dtype=np.float64)
+    rc = _get().lmo_route(ctypes.byref(cfg), x.ctypes.data, rw.ctypes.data, b.ctypes.data, n, idx.ctypes.data,
+                          w.ctypes.data)
+    if rc != 0:
+        raise ValueError("routing failed (invalid configuration)")
+    return idx, w
+
+
+def forward(cfg: LmoCfg, x, wts: dict):
+    """Full layer on the rows of x. wts: router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
+    shared_up_w, shared_down_w (bf16 as uint16). up_w/down_w are [E, ...] arrays or
+    lists of per-expert arrays (None where not needed)."""
+    x = _xarr(cfg, x)
+    n = x.shape[0]
+    keep = []
+
+    def ptr(a, dt):
+        a = _c(a, dt)
+        keep.append(a)
+        return a.ctypes.data
+
+    def expert_ptrs(arr):
+        ps = (ctypes.c_void_p * cfg.E)()
+        for e in range(cfg.E):
+            a = arr[e]
+            ps[e] = None if a is None else ptr(a, np.uint16)
+        keep.append(ps)
+        return ctypes.cast(ps, ctypes.c_void_p).value
+
+    W = LmoWeights(ptr(wts["router_w"], np.uint16), ptr(wts["e_bias"], np.float32), ptr(wts["fc1_w"], np.uint16),
+                   ptr(wts["fc2_w"], np.uint16), expert_ptrs(wts["up_w"]), expert_ptrs(wts["down_w"]),
+                   ptr(wts["shared_up_w"], np.uint16), ptr(wts["shared_down_w"], np.uint16))
+    idx = np.zeros((n, cfg.k), dtype=np.int32)
+    w = np.zeros((n, cfg.k), dtype=np.float64)
+    y = np.zeros((n, cfg.H), dtype=np.float64)
+    rc = _get().lmo_forward(ctypes.byref(cfg), x.ctypes.data, ctypes.byref(W), n, idx.ctypes.data, w.ctypes.data,
+                            y.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle forward failed (invalid configuration or missing expert weights)")
+    return y, idx, w

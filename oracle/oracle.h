@@ -1,0 +1,82 @@
+/*
+ * oracle.h -- plain, slow fp64 CPU reference of the LatentMoE layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library. It shares no code with
+ * the CUDA library and must never be used as a fallback for it.
+ *
+ * Sources (page title, section):
+ *   - "Nemotron 3 Ultra 架构 QA", Q5.1: order of the layer (fc1_latent_proj ->
+ *     experts -> fc2_latent_proj -> + shared expert on the raw input).
+ *   - same page, Q5.2: router logits = fp32 linear of the un-projected hidden
+ *     state; scores = sigmoid(logits); choice scores = scores + bias.
+ *   - same page, Q5.3: the bias is used for selection only.
+ *   - same page, Q5.7: y = fc2(sum_e w_e Expert_e(fc1(x))) + Shared(x).
+ *   - same page, Q5.8: top-k weights multiplied by routed_scaling_factor.
+ *   - same page, Q2.6: experts are non-gated, act = relu2 = max(0, x)^2.
+ *   - same page, Q5.5/Q5.6: expert weights up [E, I, L], down [E, L, I].
+ *   - "Nemotron-3-Labs-Ultra-Math-SFT" article, section "路由与共享专家":
+ *     sigmoid scoring, top-k within groups, weights normalised then x 5.0,
+ *     shared expert applied in parallel to the pre-projection input.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - group score = sum of the two largest choice scores in each contiguous
+ *     block of E/G experts; experts outside the kept groups are excluded;
+ *   - ties: tau = k-th largest eligible choice score; every expert above
+ *     tau + 1e-6 is taken, the rest come from |c - tau| <= 1e-6 in ascending
+ *     expert id (same rule for groups, with the Gk-th group score);
+ *   - normalisation divides by the plain sum of the selected sigmoid scores;
+ *   - rounding points (bf16 mode): x, z, a_e, comb and a_s are rounded to
+ *     bf16 (nearest-even) because they are GEMM operands; everything else is
+ *     fp64 here; in fp32 validation mode no rounding is applied;
+ *   - selected experts are reported in ascending expert id.
+ */
+#ifndef LMOE_ORACLE_H
+#define LMOE_ORACLE_H
+#include <stdint.h>
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+    int H, L, E, k, G, Gk, I, Is;
+    double s;       /* routed_scaling_factor */
+    int x_f32;      /* 1: x is fp32; 0: x is bf16 (uint16 bits) */
+    int fp32_mode;  /* 1: fp32 validation mode, no bf16 rounding of intermediates */
+} lmo_cfg;
+
+typedef struct {
+    const uint16_t* router_w;      /* [E, H] bf16 */
+    const float* e_bias;           /* [E] fp32 */
+    const uint16_t* fc1_w;         /* [L, H] */
+    const uint16_t* fc2_w;         /* [H, L] */
+    const uint16_t* const* up_w;   /* E pointers, each [I, L]; NULL where unused */
+    const uint16_t* const* down_w; /* E pointers, each [L, I]; NULL where unused */
+    const uint16_t* shared_up_w;   /* [Is, H] */
+    const uint16_t* shared_down_w; /* [H, Is] */
+} lmo_weights;
+
+#define LMO_EPS 1e-6
+
+/* Round to the nearest bf16 value, ties to even (exact result as a double). */
+double lmo_round_bf16(double v);
+
+/* Choice of k experts from choice scores c[E] (grouped top-k with the band
+ * rule). sel[k] receives expert ids in ascending order. Returns 0 or -1. */
+int lmo_select(const lmo_cfg* cfg, const double* c, int32_t* sel);
+
+/* Logits (fp64) for n tokens: out[t, e] = sum_h x[t, h] * W_r[e, h]. */
+int lmo_logits(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, int64_t n, double* out);
+
+/* Routing for n tokens: idx[n, k] ascending ids, w[n, k] weights. */
+int lmo_route(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, const float* e_bias, int64_t n,
+              int32_t* idx, double* w);
+
+/* Full layer for n tokens. x holds those n rows; y[n, H] fp64. idx/w may be NULL. */
+int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64_t n, int32_t* idx, double* w,
+                double* y);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
