@@ -1,0 +1,147 @@
+/*
+ * latentmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward.
+ *
+ * What the layer computes (page "Nemotron 3 Ultra 架构 QA", Q5.1, Q5.2, Q5.7,
+ * Q5.8, Q2.6; article "Nemotron-3-Labs-Ultra-Math-SFT", section
+ * "LatentMoE 层 / 路由与共享专家"):
+ *
+ *   logits = x W_r^T (fp32)          sigma = sigmoid(logits)
+ *   choice = sigma + e_score_correction_bias        (selection only)
+ *   S      = grouped top-k of choice                (n_group, topk_group, top_k)
+ *   w_e    = routed_scaling_factor * sigma_e / sum_{j in S} sigma_j
+ *   z      = x W_fc1^T                              fc1_latent_proj, H -> L
+ *   o_e    = relu(z W_up[e]^T)^2 W_down[e]^T        non-gated relu2 expert, L -> I -> L
+ *   y      = (sum_{e in S} w_e o_e) W_fc2^T + relu(x W_su^T)^2 W_sd^T
+ *
+ * Ties: tau = k-th largest eligible choice score; every expert above
+ * tau + 1e-6 is taken and the remaining slots go to |choice - tau| <= 1e-6 in
+ * ascending expert id (same rule for groups, group score = sum of the two
+ * largest choice scores of the group's E/G contiguous experts).
+ *
+ * Layouts: row-major, nn.Linear [out, in]. Expert weights are one tensor each,
+ * up [E, I, L] and down [E, L, I] (page "Nemotron 3 Ultra 架构 QA", Q5.6).
+ * All weights are bf16; e_bias is fp32. x is bf16 or fp32 ([T, H]); y is
+ * fp32 [T, H]. Every pointer is device memory owned by the caller and must be
+ * 16-byte aligned. H, L, I and Is must be multiples of 64.
+ *
+ * Modes: LMOE_MODE_BF16 feeds bf16 operands to tensor-core GEMMs with fp32
+ * accumulation (z, the expert activations, the weighted sum and the shared
+ * activations are rounded to bf16 as GEMM operands); LMOE_MODE_FP32 is a
+ * validation mode with fp32 operands and no intermediate rounding.
+ *
+ * Errors: every argument is validated before anything is launched; on
+ * LMOE_ERR_INVALID_ARG / _WORKSPACE / _UNSUPPORTED no output is touched. The
+ * library never synchronises the caller's stream and never aborts. A device
+ * wait that exceeds its bound makes the kernel record LMOE_ERR_TIMEOUT in
+ * host-visible memory and return; the call that launched it, or the next call
+ * on the handle, returns LMOE_ERR_TIMEOUT. Launch failures return
+ * LMOE_ERR_CUDA. T = 0 returns LMOE_OK and launches nothing.
+ *
+ * Determinism: the same inputs give bitwise-identical outputs (no floating-
+ * point atomics; sums run in a fixed order).
+ */
+#ifndef LATENTMOE_H
+#define LATENTMOE_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LMOE_OK = 0,
+    LMOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or shape      */
+    LMOE_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels implement        */
+    LMOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required       */
+    LMOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed      */
+    LMOE_ERR_TIMEOUT = 5,      /* a bounded device wait ran out                    */
+    LMOE_ERR_INTERNAL = 6
+} lmoe_status;
+
+typedef enum { LMOE_BF16 = 0, LMOE_FP32 = 1 } lmoe_dtype;
+typedef enum { LMOE_MODE_BF16 = 0, LMOE_MODE_FP32 = 1 } lmoe_mode;
+
+typedef struct {
+    int hidden;              /* H (multiple of 64)                               */
+    int latent;              /* L = moe_latent_size (multiple of 64)             */
+    int num_experts;         /* E = n_routed_experts                             */
+    int top_k;               /* k = num_experts_per_tok                          */
+    int n_group;             /* G; E % G == 0; G <= 32                           */
+    int topk_group;          /* Gk <= G                                          */
+    int expert_inter;        /* I = moe_intermediate_size (multiple of 64)       */
+    int shared_inter;        /* Is = moe_shared_expert_intermediate_size (x64)   */
+    int max_tokens;          /* largest T a call may pass                        */
+    float routed_scaling_factor;
+    lmoe_dtype x_dtype;      /* dtype of x                                       */
+    lmoe_mode mode;          /* BF16 (tensor cores) or FP32 (validation)         */
+} lmoe_config;
+/* Supported: E <= 1024, k <= min(64, Gk * E / G), E / G >= 2 when G > 1. */
+
+typedef struct {
+    const void* router_w;       /* [E, H]  bf16                                   */
+    const float* e_bias;        /* [E]     fp32 e_score_correction_bias           */
+    const void* fc1_w;          /* [L, H]  bf16 fc1_latent_proj                   */
+    const void* fc2_w;          /* [H, L]  bf16 fc2_latent_proj                   */
+    const void* up_w;           /* [E, I, L] bf16 expert up_proj                  */
+    const void* down_w;         /* [E, L, I] bf16 expert down_proj                */
+    const void* shared_up_w;    /* [Is, H] bf16 shared expert up_proj             */
+    const void* shared_down_w;  /* [H, Is] bf16 shared expert down_proj           */
+} lmoe_weights;
+
+typedef struct lmoe_handle lmoe_handle;
+
+/* Validates the configuration, records the (borrowed) weight pointers and
+ * pre-encodes the weight TMA descriptors. Allocates no device memory; the
+ * weights must outlive the handle. *out is set only on LMOE_OK. */
+lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out);
+
+/* Bytes of device workspace a call with T tokens needs (T <= max_tokens). */
+lmoe_status latentmoe_workspace_size(const lmoe_handle* h, int T, size_t* bytes);
+
+/* Routing only: topk_idx [T, k] int32 (ascending expert id per token),
+ * topk_w [T, k] fp32 (normalised and scaled), expert_counts [E] int32
+ * (tokens routed to each expert). Any output may be NULL. */
+lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_idx, float* topk_w,
+                            int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream);
+
+/* Full layer: y [T, H] fp32. The routing outputs are optional (NULL = not
+ * returned). ws must be at least latentmoe_workspace_size(T) bytes, 256-byte
+ * aligned, and not in use by another call in flight. */
+lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, void* ws, size_t ws_bytes,
+                              void* stream, int32_t* topk_idx, float* topk_w, int32_t* expert_counts);
+
+/* Releases the handle (host memory only). */
+void latentmoe_destroy(lmoe_handle* h);
+
+const char* latentmoe_status_string(lmoe_status s);
+
+/* ---- diagnostics --------------------------------------------------------- */
+typedef enum {
+    LMOE_OPT_GEMM_PATH = 0,      /* 0 auto, 1 tcgen05 prefill tiles, 2 tcgen05 decode (swap-AB)
+                                    tiles, 3 SIMT fp32-accumulate kernels (validation)           */
+    LMOE_OPT_ROUTER_FP64_ALL = 1,/* 1: every token's logits recomputed in fp64 (validation)      */
+    LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin for the fp64 re-check, in 1e-9 units        */
+    LMOE_OPT_SPIN_LIMIT = 3      /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */
+} lmoe_option;
+lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long value);
+
+typedef struct {
+    int flagged_tokens;     /* tokens whose routing was re-decided in fp64      */
+    int distinct_experts;   /* experts with at least one token                  */
+    int max_expert_tokens;  /* largest per-expert token count                   */
+    int device_error;       /* lmoe_status recorded by a device-side check      */
+} lmoe_stats;
+/* Reads the statistics of the last call that used ws (synchronises the device;
+ * for tests and benchmarks, not for the hot path). */
+lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out);
+
+/* Runs one kernel that waits, with the handle's spin limit, on an mbarrier
+ * that nothing ever completes, and returns the status it reports
+ * (LMOE_ERR_TIMEOUT when the bounded wait works). Synchronises the device. */
+lmoe_status latentmoe_selftest_bounded_wait(lmoe_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,216 @@
+"""Python binding of the B200 LatentMoE layer library (liblatentmoe.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. PyTorch provides device memory and the current stream. The entry
+points keep the C names (include/latentmoe.h); ``LatentMoE`` is a small
+convenience wrapper that owns a handle and a workspace.
+
+Importing this package does not load the library; the first call does, and it
+raises ``RuntimeError`` if liblatentmoe.so has not been built (there is no
+fallback implementation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblatentmoe.so")
+
+LMOE_OK, LMOE_ERR_INVALID_ARG, LMOE_ERR_UNSUPPORTED, LMOE_ERR_WORKSPACE, LMOE_ERR_CUDA, LMOE_ERR_TIMEOUT, \
+    LMOE_ERR_INTERNAL = range(7)
+LMOE_BF16, LMOE_FP32 = 0, 1
+LMOE_MODE_BF16, LMOE_MODE_FP32 = 0, 1
+OPT_GEMM_PATH, OPT_ROUTER_FP64_ALL, OPT_FLAG_DELTA, OPT_SPIN_LIMIT = range(4)
+GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
+
+EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
+           "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
+           "latentmoe_selftest_bounded_wait"]
+
+
+class lmoe_config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("latent", ctypes.c_int), ("num_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int),
+                ("expert_inter", ctypes.c_int), ("shared_inter", ctypes.c_int), ("max_tokens", ctypes.c_int),
+                ("routed_scaling_factor", ctypes.c_float), ("x_dtype", ctypes.c_int), ("mode", ctypes.c_int)]
+
+
+class lmoe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
+                                                "shared_up_w", "shared_down_w")]
+
+
+class lmoe_stats(ctypes.Structure):
+    _fields_ = [("flagged_tokens", ctypes.c_int), ("distinct_experts", ctypes.c_int),
+                ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int)]
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+_lib = None
+
+
+def load():
+    """Load liblatentmoe.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("liblatentmoe.so is not built (run `python -c 'import __graft_entry__ as g; g.build()'`); "
+                           "the LatentMoE layer has no non-CUDA implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.latentmoe_create.argtypes = [ctypes.POINTER(lmoe_config), ctypes.POINTER(lmoe_weights), ctypes.POINTER(vp)]
+    lib.latentmoe_workspace_size.argtypes = [vp, i32, ctypes.POINTER(sz)]
+    lib.latentmoe_route.argtypes = [vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.latentmoe_forward.argtypes = [vp, vp, i32, vp, vp, sz, vp, vp, vp, vp]
+    lib.latentmoe_destroy.argtypes = [vp]
+    lib.latentmoe_destroy.restype = None
+    lib.latentmoe_status_string.argtypes = [i32]
+    lib.latentmoe_status_string.restype = ctypes.c_char_p
+    lib.latentmoe_set_option.argtypes = [vp, i32, ctypes.c_longlong]
+    lib.latentmoe_read_stats.argtypes = [vp, vp, ctypes.POINTER(lmoe_stats)]
+    lib.latentmoe_selftest_bounded_wait.argtypes = [vp]
+    for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
+              "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait"):
+        getattr(lib, f).restype = i32
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load().latentmoe_status_string(int(s)).decode()
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+# ---------------------------------------------------------------- C entry points
+def latentmoe_create(cfg: lmoe_config, w: lmoe_weights):
+    h = ctypes.c_void_p()
+    s = load().latentmoe_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
+    return s, h
+
+
+def latentmoe_workspace_size(h, T: int):
+    n = ctypes.c_size_t()
+    s = load().latentmoe_workspace_size(h, T, ctypes.byref(n))
+    return s, n.value
+
+
+def latentmoe_route(h, x, T, idx, w, counts, ws, ws_bytes, stream):
+    return load().latentmoe_route(h, x, T, idx, w, counts, ws, ws_bytes, stream)
+
+
+def latentmoe_forward(h, x, T, y, ws, ws_bytes, stream, idx=None, w=None, counts=None):
+    return load().latentmoe_forward(h, x, T, y, ws, ws_bytes, stream, idx, w, counts)
+
+
+def latentmoe_destroy(h):
+    load().latentmoe_destroy(h)
+
+
+def latentmoe_set_option(h, opt: int, value: int) -> int:
+    return load().latentmoe_set_option(h, opt, value)
+
+
+def latentmoe_read_stats(h, ws):
+    st = lmoe_stats()
+    s = load().latentmoe_read_stats(h, ws, ctypes.byref(st))
+    return s, st
+
+
+def latentmoe_selftest_bounded_wait(h) -> int:
+    return load().latentmoe_selftest_bounded_wait(h)
+
+
+# ---------------------------------------------------------------- convenience wrapper
+class LatentMoE:
+    """A handle plus a workspace, driven with torch tensors.
+
+    shape: an object with H, L, E, k, G, Gk, I, Is, s (e.g. synth.LayerShape).
+    weights: dict of CUDA tensors router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
+    shared_up_w, shared_down_w (bf16, e_bias fp32). The tensors are borrowed.
+    """
+
+    def __init__(self, shape, weights: dict, max_tokens: int, x_f32: bool = False, mode: int = LMOE_MODE_BF16):
+        import torch
+        self.torch = torch
+        self.shape = shape
+        self.weights = weights
+        cfg = lmoe_config(shape.H, shape.L, shape.E, shape.k, shape.G, shape.Gk, shape.I, shape.Is, max_tokens,
+                          float(shape.s), LMOE_FP32 if x_f32 else LMOE_BF16, mode)
+        w = lmoe_weights(*[_p(weights[n]) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
+                                                     "shared_up_w", "shared_down_w")])
+        s, h = latentmoe_create(cfg, w)
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_create")
+        self.h = h
+        self.cfg = cfg
+        self.x_f32 = x_f32
+        self.mode = mode
+        self._ws = None
+        self._ws_T = -1
+
+    def workspace(self, T: int):
+        s, n = latentmoe_workspace_size(self.h, T)
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_workspace_size")
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = self.torch.empty(max(n, 256), dtype=self.torch.uint8, device="cuda")
+        return self._ws, n
+
+    def set_option(self, opt: int, value: int):
+        s = latentmoe_set_option(self.h, opt, value)
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_set_option")
+
+    def _stream(self):
+        return ctypes.c_void_p(self.torch.cuda.current_stream().cuda_stream)
+
+    def forward(self, x, y=None, idx=None, w=None, counts=None):
+        torch = self.torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.shape.H), dtype=torch.float32, device=x.device)
+        ws, n = self.workspace(T)
+        s = latentmoe_forward(self.h, _p(x), T, _p(y), _p(ws), ws.numel(), self._stream(), _p(idx), _p(w), _p(counts))
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_forward")
+        return y
+
+    def route(self, x, idx=None, w=None, counts=None):
+        torch = self.torch
+        T = x.shape[0]
+        k, E = self.shape.k, self.shape.E
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx is None else idx
+        w = torch.empty((T, k), dtype=torch.float32, device=x.device) if w is None else w
+        counts = torch.empty((E,), dtype=torch.int32, device=x.device) if counts is None else counts
+        ws, n = self.workspace(T)
+        s = latentmoe_route(self.h, _p(x), T, _p(idx), _p(w), _p(counts), _p(ws), ws.numel(), self._stream())
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_route")
+        return idx, w, counts
+
+    def stats(self):
+        s, st = latentmoe_read_stats(self.h, _p(self._ws))
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_read_stats")
+        return st
+
+    def close(self):
+        if getattr(self, "h", None):
+            latentmoe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

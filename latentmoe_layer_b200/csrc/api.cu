@@ -1,0 +1,497 @@
+// api.cpp -- the C ABI of the LatentMoE layer forward (include/latentmoe.h):
+// argument validation, workspace carving, TMA descriptor encoding and the
+// launch sequence. Every launch goes to the caller's stream; nothing here
+// synchronises except the diagnostic entry points that say so.
+//
+// Launch sequence of latentmoe_forward (bf16 mode):
+//   1 router GEMM       logits = x W_r^T (fp32, tensor cores)
+//   2 select            sigmoid, +bias, grouped top-k, weights; near-edge flags
+//   3 fp64 re-check     flagged tokens: exact-product fp64 logits and decision
+//   4 permutation       counts, offsets, tile prefixes, perm, slot, row weights
+//   5 input GEMM        z = x W_fc1^T (bf16) and a_s = relu2(x W_su^T) (bf16)
+//   6 gather            z rows into expert order
+//   7 expert up GEMM    a = relu2(z_e W_up[e]^T) (bf16), grouped by expert
+//   8 expert down GEMM  o = w * (a_e W_down[e]^T) (fp32), grouped by expert
+//   9 combine           comb[t] = bf16(sum over the token's k rows, ascending id)
+//  10 output GEMM       y = comb W_fc2^T + a_s W_sd^T (fp32), one K-concatenated GEMM
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "handle.h"
+#include "lmoe_internal.h"
+
+using namespace lmoe;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+
+bool get_encoder() {
+    if (g_encode) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return true;
+}
+
+// bf16 row-major [rows, cols] with cols contiguous; box = 64 columns (one
+// 128-byte swizzle row) x box_rows rows.
+bool encode_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+bool plan_of(const lmoe_config& c, int T, Plan& p) {
+    const size_t E = c.num_experts, k = c.top_k, H = c.hidden, L = c.latent, I = c.expert_inter,
+                 Is = c.shared_inter;
+    const size_t A = (size_t)T * k;
+    const size_t act = c.mode == LMOE_MODE_BF16 ? 2 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += al256(bytes);
+        return o;
+    };
+    p.T = T;
+    p.A = (int)A;
+    p.nblk = (T + 255) / 256;
+    p.stats = take(sizeof(WsStats));
+    p.logits = take((size_t)T * E * 4);
+    p.logits64 = take((size_t)T * E * 8);
+    p.flaglist = take((size_t)T * 4);
+    p.idx = take(A * 4);
+    p.wgt = take(A * 4);
+    p.counts = take(E * 4);
+    p.offsets = take((E + 1) * 4);
+    p.pfx128 = take((E + 1) * 4);
+    p.pfx64 = take((E + 1) * 4);
+    p.pfxdec = take((E + 1) * 4);
+    p.blockcounts = take((size_t)p.nblk * E * 4);
+    p.perm = take(A * 4);
+    p.slot = take(A * 4);
+    p.wperm = take(A * 4);
+    p.xbf = (c.mode == LMOE_MODE_BF16 && c.x_dtype == LMOE_FP32) ? take((size_t)T * H * 2) : 0;
+    p.z = take((size_t)T * L * act);
+    p.zperm = take(A * L * act);
+    p.aperm = take(A * I * act);
+    p.o = take(A * L * 4);
+    p.comb = take((size_t)T * L * act);
+    p.as = take((size_t)T * Is * act);
+    p.total = off;
+    return true;
+}
+
+lmoe_status check_config(const lmoe_config* c) {
+    if (!c) return LMOE_ERR_INVALID_ARG;
+    if (c->hidden <= 0 || c->latent <= 0 || c->num_experts <= 0 || c->top_k <= 0 || c->n_group <= 0 ||
+        c->topk_group <= 0 || c->expert_inter <= 0 || c->shared_inter <= 0 || c->max_tokens <= 0)
+        return LMOE_ERR_INVALID_ARG;
+    if (c->hidden % 64 || c->latent % 64 || c->expert_inter % 64 || c->shared_inter % 64)
+        return LMOE_ERR_INVALID_ARG;
+    if (c->num_experts % c->n_group || c->topk_group > c->n_group) return LMOE_ERR_INVALID_ARG;
+    if (c->top_k > c->topk_group * (c->num_experts / c->n_group)) return LMOE_ERR_INVALID_ARG;
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor) || isinf(c->routed_scaling_factor))
+        return LMOE_ERR_INVALID_ARG;
+    if ((c->x_dtype != LMOE_BF16 && c->x_dtype != LMOE_FP32) ||
+        (c->mode != LMOE_MODE_BF16 && c->mode != LMOE_MODE_FP32))
+        return LMOE_ERR_INVALID_ARG;
+    if (c->num_experts > kMaxE || c->n_group > kMaxG || c->top_k > kMaxK) return LMOE_ERR_UNSUPPORTED;
+    if (c->n_group > 1 && c->num_experts / c->n_group < 2) return LMOE_ERR_UNSUPPORTED;
+    if (c->hidden > 16384) return LMOE_ERR_UNSUPPORTED;  // fp64 router stages one x row in shared memory
+    if ((long long)c->max_tokens * c->top_k > (1LL << 30)) return LMOE_ERR_UNSUPPORTED;
+    return LMOE_OK;
+}
+
+lmoe_status check_weights(const lmoe_weights* w) {
+    if (!w) return LMOE_ERR_INVALID_ARG;
+    const void* ps[8] = {w->router_w, w->e_bias, w->fc1_w, w->fc2_w, w->up_w, w->down_w, w->shared_up_w,
+                         w->shared_down_w};
+    for (const void* p : ps)
+        if (!p || !aligned(p, 16)) return LMOE_ERR_INVALID_ARG;
+    return LMOE_OK;
+}
+
+// Tensor-core tile choice for a set of problem widths.
+int pick_bn(const int* ns, int cnt) {
+    for (int bn : {256, 128, 64}) {
+        bool ok = true;
+        for (int i = 0; i < cnt; ++i) ok = ok && ns[i] % bn == 0;
+        if (ok) return bn;
+    }
+    return 0;
+}
+
+struct Ctx {
+    lmoe_handle* h;
+    const Plan* p;
+    char* ws;
+    cudaStream_t s;
+    DeviceRouting r;
+    int* err;
+    bool decode;  // swap-AB tiles for the expert GEMMs and the dense GEMMs
+    bool simt;
+};
+
+// Runs one GEMM launch (1 or 2 problems sharing the tile path). Operands are
+// given as (pointer, rows, K) and encoded here for the chosen tile shape.
+struct Operand {
+    const void* ptr;
+    long long rows;
+};
+
+cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2], const Operand (*b)[2],
+                     bool a_f32_simt) {
+    if (c.simt) return launch_gemm_simt(probs, nprob, a_f32_simt, c.r, c.p->A, c.s);
+    int ns[2] = {probs[0].n, nprob > 1 ? probs[1].n : probs[0].n};
+    bool swap = c.decode;
+    for (int i = 0; i < nprob; ++i) swap = swap && probs[i].n % 128 == 0;
+    const int bn = swap ? kDecodeTN : pick_bn(ns, nprob);
+    if (bn == 0) return cudaErrorInvalidValue;
+    CUtensorMap maps[8];
+    int nm = 0;
+    for (int i = 0; i < nprob; ++i)
+        for (int sg = 0; sg < probs[i].nseg; ++sg) {
+            const int K = probs[i].kdim[sg];
+            if (!encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? kDecodeTN : kBM))
+                return cudaErrorInvalidValue;
+            probs[i].a_map[sg] = nm++;
+            if (!encode_bf16(&maps[nm], b[i][sg].ptr, b[i][sg].rows, K, swap ? kBM : bn))
+                return cudaErrorInvalidValue;
+            probs[i].b_map[sg] = nm++;
+        }
+    if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
+    return launch_gemm_tc(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
+}
+
+GemmProblem make_problem(int grouped, int m_rows, int n, int epi, void* out, long long ldo) {
+    GemmProblem p;
+    memset(&p, 0, sizeof(p));
+    p.grouped = grouped;
+    p.m_rows = m_rows;
+    p.n = n;
+    p.nseg = 1;
+    p.epi = epi;
+    p.out = out;
+    p.ldo = ldo;
+    return p;
+}
+
+lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA; }
+
+#define LMOE_TRY(expr)                                   \
+    do {                                                 \
+        cudaError_t _e = (expr);                         \
+        if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
+    } while (0)
+
+__attribute__((unused)) lmoe_status take_device_error(lmoe_handle* h) {
+    volatile int* he = h->herr;
+    int v = *he;
+    if (v != 0) {
+        *he = 0;
+        return (lmoe_status)v;
+    }
+    return LMOE_OK;
+}
+
+lmoe_status validate_call(lmoe_handle* h, const void* x, int T, void* ws, size_t ws_bytes, Plan& p) {
+    if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!x || !aligned(x, 16)) return LMOE_ERR_INVALID_ARG;
+    plan_of(h->cfg, T, p);
+    if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return LMOE_ERR_WORKSPACE;
+    return LMOE_OK;
+}
+
+// Routing stages 1-4. Writes idx/w/counts into the workspace and, if given,
+// the caller's outputs.
+lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const Plan& p = *c.p;
+    char* ws = c.ws;
+    const bool fp64_all = h->fp64_all || cf.mode == LMOE_MODE_FP32 || cf.x_dtype == LMOE_FP32 ||
+                          cf.num_experts % 64 != 0 || c.simt;
+    LMOE_TRY(cudaMemsetAsync(ws + p.stats, 0, sizeof(WsStats), c.s));
+    if (!fp64_all) {
+        GemmProblem pr = make_problem(0, p.T, cf.num_experts, EPI_F32, ws + p.logits, cf.num_experts);
+        pr.kdim[0] = cf.hidden;
+        Operand a[1][2] = {{{x, p.T}, {nullptr, 0}}};
+        Operand b[1][2] = {{{h->w.router_w, cf.num_experts}, {nullptr, 0}}};
+        Ctx rc = c;
+        rc.decode = c.decode && cf.num_experts % 128 == 0;
+        LMOE_TRY(run_gemm(rc, &pr, 1, a, b, false));
+        LMOE_TRY(launch_router_select(h, p, ws, false, c.s));
+        LMOE_TRY(launch_router_logits64(h, x, p, ws, false, c.s));
+        LMOE_TRY(launch_router_select64(h, p, ws, false, c.s));
+    } else {
+        LMOE_TRY(launch_router_logits64(h, x, p, ws, true, c.s));
+        LMOE_TRY(launch_router_select64(h, p, ws, true, c.s));
+    }
+    LMOE_TRY(launch_permute(h, p, ws, counts_out, c.s));
+    LMOE_TRY(launch_copy_routing(reinterpret_cast<const int*>(ws + p.idx), reinterpret_cast<const float*>(ws + p.wgt),
+                                 idx_out, w_out, (long long)p.T * cf.top_k, c.s));
+    return LMOE_OK;
+}
+
+Ctx make_ctx(lmoe_handle* h, const Plan& p, void* ws, void* stream) {
+    Ctx c;
+    c.h = h;
+    c.p = &p;
+    c.ws = static_cast<char*>(ws);
+    c.s = static_cast<cudaStream_t>(stream);
+    c.r.offsets = reinterpret_cast<const int*>(c.ws + p.offsets);
+    c.r.pfx128 = reinterpret_cast<const int*>(c.ws + p.pfx128);
+    c.r.pfx64 = reinterpret_cast<const int*>(c.ws + p.pfx64);
+    c.r.pfxdec = reinterpret_cast<const int*>(c.ws + p.pfxdec);
+    c.r.E = h->cfg.num_experts;
+    c.err = &reinterpret_cast<WsStats*>(c.ws + p.stats)->device_error;
+    const lmoe_config& cf = h->cfg;
+    c.simt = h->gemm_path == 3 || cf.mode == LMOE_MODE_FP32;
+    if (h->gemm_path == 1) c.decode = false;
+    else if (h->gemm_path == 2) c.decode = true;
+    else c.decode = (long long)p.T * cf.top_k <= 64LL * cf.num_experts;  // <= 64 rows per expert on average
+    return c;
+}
+
+__global__ void k_publish_error(const int* derr, int* herr) {
+    int v = *derr;
+    if (v != 0) *(volatile int*)herr = v;
+}
+
+}  // namespace
+
+extern "C" {
+
+lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out) {
+    if (!out) return LMOE_ERR_INVALID_ARG;
+    lmoe_status s = check_config(cfg);
+    if (s != LMOE_OK) return s;
+    s = check_weights(w);
+    if (s != LMOE_OK) return s;
+    if (!get_encoder()) return LMOE_ERR_CUDA;
+    lmoe_handle* h = new (std::nothrow) lmoe_handle();
+    if (!h) return LMOE_ERR_INTERNAL;
+    h->cfg = *cfg;
+    h->w = *w;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&h->herr), 64, cudaHostAllocMapped) != cudaSuccess) {
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    *h->herr = 0;
+    if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->derr), h->herr, 0) != cudaSuccess) {
+        cudaFreeHost(h->herr);
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    h->num_sms = tc_num_sms();
+    *out = h;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_workspace_size(const lmoe_handle* h, int T, size_t* bytes) {
+    if (!h || !bytes || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    Plan p;
+    plan_of(h->cfg, T, p);
+    *bytes = T == 0 ? 0 : p.total;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_idx, float* topk_w,
+                            int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+        (expert_counts && !aligned(expert_counts, 4)))
+        return LMOE_ERR_INVALID_ARG;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    Ctx c = make_ctx(h, p, ws, stream);
+    s = do_route(c, x, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    return cuda_status(cudaGetLastError());
+}
+
+lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, void* ws, size_t ws_bytes,
+                              void* stream, int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    if (!y || !aligned(y, 16)) return LMOE_ERR_INVALID_ARG;
+    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+        (expert_counts && !aligned(expert_counts, 4)))
+        return LMOE_ERR_INVALID_ARG;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    const lmoe_config& cf = h->cfg;
+    Ctx c = make_ctx(h, p, ws, stream);
+    char* ws_c = c.ws;
+    s = do_route(c, x, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
+
+    const bool bf16 = cf.mode == LMOE_MODE_BF16;
+    const int act = bf16 ? 2 : 4;
+    const int H = cf.hidden, L = cf.latent, I = cf.expert_inter, Is = cf.shared_inter, E = cf.num_experts;
+    const long long A = p.A;
+    // GEMM operand x: bf16 x as given, fp32 x rounded to bf16 (bf16 mode) or fp32 x (validation mode).
+    const void* xa = x;
+    bool xa_f32 = cf.x_dtype == LMOE_FP32;
+    if (bf16 && cf.x_dtype == LMOE_FP32) {
+        LMOE_TRY(launch_convert_x(static_cast<const float*>(x), reinterpret_cast<uint16_t*>(ws_c + p.xbf),
+                                  (long long)p.T * H, c.s));
+        xa = ws_c + p.xbf;
+        xa_f32 = false;
+    }
+    const int epi_act = bf16 ? EPI_BF16 : EPI_F32;
+    const int epi_relu2 = bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32;
+
+    // 5: z = x W_fc1^T, a_s = relu2(x W_su^T)
+    {
+        GemmProblem pr[2] = {make_problem(0, p.T, L, epi_act, ws_c + p.z, L),
+                             make_problem(0, p.T, Is, epi_relu2, ws_c + p.as, Is)};
+        pr[0].kdim[0] = H;
+        pr[1].kdim[0] = H;
+        pr[0].a_ptr[0] = xa;
+        pr[0].b_ptr[0] = h->w.fc1_w;
+        pr[1].a_ptr[0] = xa;
+        pr[1].b_ptr[0] = h->w.shared_up_w;
+        Operand a[2][2] = {{{xa, p.T}, {nullptr, 0}}, {{xa, p.T}, {nullptr, 0}}};
+        Operand b[2][2] = {{{h->w.fc1_w, L}, {nullptr, 0}}, {{h->w.shared_up_w, Is}, {nullptr, 0}}};
+        LMOE_TRY(run_gemm(c, pr, 2, a, b, xa_f32));
+    }
+    // 6: expert-ordered copy of z
+    LMOE_TRY(launch_gather_rows(ws_c + p.z, ws_c + p.zperm, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
+                                reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
+    // 7: a = relu2(z_e W_up[e]^T)
+    {
+        GemmProblem pr = make_problem(1, 0, I, epi_relu2, ws_c + p.aperm, I);
+        pr.kdim[0] = L;
+        pr.b_rows_per_expert = I;
+        pr.a_ptr[0] = ws_c + p.zperm;
+        pr.b_ptr[0] = h->w.up_w;
+        Operand a[1][2] = {{{ws_c + p.zperm, A}, {nullptr, 0}}};
+        Operand b[1][2] = {{{h->w.up_w, (long long)E * I}, {nullptr, 0}}};
+        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+    }
+    // 8: o = w * (a_e W_down[e]^T)
+    {
+        GemmProblem pr = make_problem(1, 0, L, EPI_SCALE_F32, ws_c + p.o, L);
+        pr.kdim[0] = I;
+        pr.b_rows_per_expert = L;
+        pr.row_scale = reinterpret_cast<const float*>(ws_c + p.wperm);
+        pr.a_ptr[0] = ws_c + p.aperm;
+        pr.b_ptr[0] = h->w.down_w;
+        Operand a[1][2] = {{{ws_c + p.aperm, A}, {nullptr, 0}}};
+        Operand b[1][2] = {{{h->w.down_w, (long long)E * L}, {nullptr, 0}}};
+        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+    }
+    // 9: comb
+    LMOE_TRY(launch_combine(reinterpret_cast<const float*>(ws_c + p.o), reinterpret_cast<const int*>(ws_c + p.slot),
+                            ws_c + p.comb, p.T, cf.top_k, L, bf16, c.s));
+    // 10: y = comb W_fc2^T + a_s W_sd^T
+    {
+        GemmProblem pr = make_problem(0, p.T, H, EPI_F32, y, H);
+        pr.nseg = 2;
+        pr.kdim[0] = L;
+        pr.kdim[1] = Is;
+        pr.a_ptr[0] = ws_c + p.comb;
+        pr.b_ptr[0] = h->w.fc2_w;
+        pr.a_ptr[1] = ws_c + p.as;
+        pr.b_ptr[1] = h->w.shared_down_w;
+        Operand a[1][2] = {{{ws_c + p.comb, p.T}, {ws_c + p.as, p.T}}};
+        Operand b[1][2] = {{{h->w.fc2_w, H}, {h->w.shared_down_w, H}}};
+        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+    }
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    return cuda_status(cudaGetLastError());
+}
+
+void latentmoe_destroy(lmoe_handle* h) {
+    if (!h) return;
+    if (h->herr) cudaFreeHost(h->herr);
+    delete h;
+}
+
+const char* latentmoe_status_string(lmoe_status s) {
+    switch (s) {
+        case LMOE_OK: return "ok";
+        case LMOE_ERR_INVALID_ARG: return "invalid argument";
+        case LMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case LMOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case LMOE_ERR_CUDA: return "CUDA error";
+        case LMOE_ERR_TIMEOUT: return "bounded device wait timed out";
+        case LMOE_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
+    if (!h) return LMOE_ERR_INVALID_ARG;
+    switch (opt) {
+        case LMOE_OPT_GEMM_PATH:
+            if (v < 0 || v > 3) return LMOE_ERR_INVALID_ARG;
+            h->gemm_path = (int)v;
+            return LMOE_OK;
+        case LMOE_OPT_ROUTER_FP64_ALL:
+            h->fp64_all = v != 0;
+            return LMOE_OK;
+        case LMOE_OPT_FLAG_DELTA:
+            if (v < 0 || v > 100000000) return LMOE_ERR_INVALID_ARG;
+            h->flag_delta = (float)(v * 1e-9);
+            return LMOE_OK;
+        case LMOE_OPT_SPIN_LIMIT:
+            if (v < 1 || v > 0xFFFFFFFFLL) return LMOE_ERR_INVALID_ARG;
+            h->spin_limit = (unsigned)v;
+            return LMOE_OK;
+    }
+    return LMOE_ERR_INVALID_ARG;
+}
+
+lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out) {
+    if (!h || !ws || !out) return LMOE_ERR_INVALID_ARG;
+    WsStats st;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+    out->flagged_tokens = st.flagged;
+    out->distinct_experts = st.distinct;
+    out->max_expert_tokens = st.max_count;
+    out->device_error = st.device_error;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_selftest_bounded_wait(lmoe_handle* h) {
+    if (!h) return LMOE_ERR_INVALID_ARG;
+    int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) return LMOE_ERR_CUDA;
+    int v = 0;
+    cudaError_t e = cudaMemset(d, 0, sizeof(int));
+    if (e == cudaSuccess) e = launch_selftest_wait(d, h->spin_limit, 0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&v, d, sizeof(int), cudaMemcpyDeviceToHost);
+    cudaFree(d);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    return (lmoe_status)v;
+}
+
+}  // extern "C"

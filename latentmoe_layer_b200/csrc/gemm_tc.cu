@@ -1,0 +1,455 @@
+// gemm_tc.cu -- persistent tcgen05 GEMM engine for sm_100a.
+//
+// Every dense contraction of the layer runs here: the router logits, fc1
+// (fc1_latent_proj), the shared expert's up projection, each routed expert's
+// up and down projection (grouped by expert over the permuted rows) and the
+// output GEMM that fuses fc2_latent_proj with the shared expert's down
+// projection by concatenating their K ranges into one accumulator
+// (y = comb W_fc2^T + a_s W_sd^T; "Nemotron 3 Ultra 架构 QA", Q5.7).
+//
+// Structure of one CTA (one per SM, persistent over tiles):
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles into a ring of
+//               shared-memory stages (mbarrier complete_tx), no multicast.
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.cta_group::1.kind::f16
+//               128 x BN x 16 per instruction, fp32 accumulators in TMEM,
+//               double-buffered so the epilogue of tile i overlaps tile i+1.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, the fused
+//               activation (relu2), weight scaling or bf16 rounding, stores.
+//
+// Two tile shapes share the code:
+//   kSwap = false  MMA M = 128 activation rows, N = BN weight rows.
+//   kSwap = true   MMA M = 128 weight rows, N = BN tokens (decode batches,
+//                  where each expert sees a handful of tokens: the weights sit
+//                  on the 128-row side so no tensor-core work is padding).
+// Every mbarrier wait is bounded; on running out the kernel records
+// LMOE_ERR_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and returns.
+#include <cuda_bf16.h>
+#include <string.h>
+
+#include "lmoe_internal.h"
+#include "ptx.cuh"
+
+namespace lmoe {
+namespace {
+
+constexpr int kMaxMaps = 8;
+constexpr int kThreads = 192;
+constexpr int kGroupM = 16;
+
+struct alignas(64) TcParams {
+    CUtensorMap maps[kMaxMaps];
+    GemmProblem prob[2];
+    int nprob;
+    int nmaps;
+    int dense_tiles[2];
+    DeviceRouting r;
+    int* err;
+    unsigned spin;
+};
+
+struct TileInfo {
+    int p;       // problem
+    int row0;    // first activation row (permuted row for grouped problems)
+    int rows;    // valid activation rows in this tile
+    int wrow0;   // first weight row (row of B)
+    int col0;    // first output column
+};
+
+template <int BN, bool kSwap>
+struct Shape {
+    static constexpr int XR = 128;            // rows of the MMA A operand tile
+    static constexpr int YR = BN;             // rows of the MMA B operand tile
+    static constexpr int kXBytes = XR * kBK * 2;
+    static constexpr int kYBytes = YR * kBK * 2;
+    static constexpr int kStageBytes = kXBytes + kYBytes;
+    static constexpr int kActRows = kSwap ? BN : 128;   // activation rows per tile
+    static constexpr int kOutCols = kSwap ? 128 : BN;   // output columns per tile
+    static constexpr uint32_t kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+};
+
+__device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
+
+template <int BN, bool kSwap>
+__device__ __forceinline__ int total_tiles(const TcParams& P) {
+    using S = Shape<BN, kSwap>;
+    if (P.prob[0].grouped) {
+        const int* pfx = kSwap ? P.r.pfxdec : P.r.pfx128;
+        return pfx[P.r.E] * n_col_tiles(P.prob[0], S::kOutCols);
+    }
+    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
+}
+
+// Tile t -> coordinates. Dense problems are rasterised in groups of kGroupM
+// row tiles (column tiles outer within a group) so that concurrently running
+// CTAs share both operands in L2. Grouped problems walk experts in order,
+// column tiles inner, so an expert's weights are read while its rows are hot.
+template <int BN, bool kSwap>
+__device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
+    using S = Shape<BN, kSwap>;
+    TileInfo ti;
+    if (P.prob[0].grouped) {
+        const GemmProblem& pr = P.prob[0];
+        const int nct = n_col_tiles(pr, S::kOutCols);
+        const int mt = t / nct, ct = t % nct;
+        const int* pfx = kSwap ? P.r.pfxdec : P.r.pfx128;
+        int lo = 0, hi = P.r.E;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (__ldg(&pfx[mid]) <= mt) lo = mid;
+            else hi = mid;
+        }
+        const int e = lo;
+        const int off = __ldg(&P.r.offsets[e]), end = __ldg(&P.r.offsets[e + 1]);
+        ti.p = 0;
+        ti.row0 = off + (mt - __ldg(&pfx[e])) * S::kActRows;
+        ti.rows = min(S::kActRows, end - ti.row0);
+        ti.col0 = ct * S::kOutCols;
+        ti.wrow0 = e * pr.b_rows_per_expert + ti.col0;
+        return ti;
+    }
+    int p = 0;
+    if (P.nprob > 1 && t >= P.dense_tiles[0]) {
+        t -= P.dense_tiles[0];
+        p = 1;
+    }
+    const GemmProblem& pr = P.prob[p];
+    const int nct = n_col_tiles(pr, S::kOutCols);
+    const int mtc = (pr.m_rows + S::kActRows - 1) / S::kActRows;
+    int mt, ct;
+    if (kSwap) {  // token tiles inner: the tiles that share a weight block run together
+        ct = t / mtc;
+        mt = t % mtc;
+    } else {
+        const int g = t / (kGroupM * nct), r = t % (kGroupM * nct);
+        const int ms = min(kGroupM, mtc - g * kGroupM);
+        mt = g * kGroupM + r % ms;
+        ct = r / ms;
+    }
+    ti.p = p;
+    ti.row0 = mt * S::kActRows;
+    ti.rows = min(S::kActRows, pr.m_rows - ti.row0);
+    ti.col0 = ct * S::kOutCols;
+    ti.wrow0 = ti.col0;
+    return ti;
+}
+
+template <int BN, bool kSwap>
+__device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const TileInfo& ti, int lane_row, int c0,
+                                               const uint32_t (&r)[16]) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+    const int epi = pr.epi;
+    if (epi == EPI_RELU2_BF16 || epi == EPI_RELU2_F32) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float a = fmaxf(v[i], 0.f);
+            v[i] = a * a;
+        }
+    }
+    if (!kSwap) {
+        // thread owns activation row (row0 + lane_row), columns col0 + c0 .. +15
+        if (lane_row >= ti.rows) return;
+        const long long row = ti.row0 + lane_row;
+        if (epi == EPI_SCALE_F32) {
+            const float s = __ldg(&pr.row_scale[row]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= s;
+        }
+        if (epi == EPI_BF16 || epi == EPI_RELU2_BF16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) + row * pr.ldo + ti.col0 + c0);
+            dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                pack_bf16x2(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                pack_bf16x2(v[14], v[15]));
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + row * pr.ldo + ti.col0 + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+    } else {
+        // thread owns output column (col0 + lane_row); columns of the
+        // accumulator are tokens row0 + c0 .. +15.
+        const long long col = ti.col0 + lane_row;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int tok = c0 + i;
+            if (tok < ti.rows) {
+                const long long row = ti.row0 + tok;
+                float x = v[i];
+                if (epi == EPI_SCALE_F32) x *= __ldg(&pr.row_scale[row]);
+                if (epi == EPI_BF16 || epi == EPI_RELU2_BF16)
+                    static_cast<__nv_bfloat16*>(pr.out)[row * pr.ldo + col] = __float2bfloat16_rn(x);
+                else
+                    static_cast<float*>(pr.out)[row * pr.ldo + col] = x;
+            }
+        }
+    }
+}
+
+template <int BN, int STAGES, bool kSwap>
+__global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+    using S = Shape<BN, kSwap>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base_u32 = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
+    uint8_t* sX = smem;                                  // STAGES x kXBytes
+    uint8_t* sY = smem + STAGES * S::kXBytes;            // STAGES x kYBytes
+    uint64_t* full = reinterpret_cast<uint64_t*>(sY + STAGES * S::kYBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, S::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntiles = total_tiles<BN, kSwap>(P);
+    int* err = P.err;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0, issued = 0, issued_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, kSwap>(P, t);
+            const GemmProblem& pr = P.prob[ti.p];
+            for (int sg = 0; sg < pr.nseg && ok; ++sg) {
+                const CUtensorMap* amap = &P.maps[pr.a_map[sg]];
+                const CUtensorMap* bmap = &P.maps[pr.b_map[sg]];
+                const int kb_n = pr.kdim[sg] / kBK;
+                for (int kb = 0; kb < kb_n; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, P.spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    if (!kSwap) {
+                        tma_load_2d(sX + stage * S::kXBytes, amap, &full[stage], kb * kBK, ti.row0);
+                        tma_load_2d(sY + stage * S::kYBytes, bmap, &full[stage], kb * kBK, ti.wrow0);
+                    } else {
+                        tma_load_2d(sX + stage * S::kXBytes, bmap, &full[stage], kb * kBK, ti.wrow0);
+                        tma_load_2d(sY + stage * S::kYBytes, amap, &full[stage], kb * kBK, ti.row0);
+                    }
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        // every load this thread issued has landed before the CTA can exit
+        for (int s = 0; s < STAGES; ++s)
+            if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, kSwap>(P, t);
+            const GemmProblem& pr = P.prob[ti.p];
+            if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, P.spin, err)) break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+            uint32_t accumulate = 0;
+            for (int sg = 0; sg < pr.nseg && ok; ++sg) {
+                const int kb_n = pr.kdim[sg] / kBK;
+                for (int kb = 0; kb < kb_n; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_sw128(smem_u32(sX + stage * S::kXBytes));
+                    const uint64_t bdesc = sdesc_sw128(smem_u32(sY + stage * S::kYBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        // +32 bytes per K step of 16 bf16 inside the 128-byte swizzled row
+                        umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, accumulate);
+                        accumulate = 1;
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) break;
+            umma_commit(&tfull[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        // all MMAs issued by this thread have completed before TMEM is freed
+        umma_commit(done);
+        mbar_wait_bounded(done, 0, 1u << 26, err);
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int lane_row = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, kSwap>(P, t);
+            const GemmProblem& pr = P.prob[ti.p];
+            if (!mbar_wait_bounded(&tfull[acc], acc_phase, P.spin, err)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(taddr + (uint32_t)c0, r);
+                tmem_ld_wait();
+                epilogue_store<BN, kSwap>(pr, ti, lane_row, c0, r);
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+}
+
+template <int BN, int STAGES, bool kSwap>
+constexpr size_t smem_bytes() {
+    return 1024 + (size_t)STAGES * Shape<BN, kSwap>::kStageBytes + 256;
+}
+
+template <int BN, int STAGES, bool kSwap>
+cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
+    constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
+    static_assert(smem <= 232448, "shared memory");
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    k_gemm_tc<BN, STAGES, kSwap><<<grid, kThreads, smem, s>>>(P);
+    return cudaGetLastError();
+}
+
+int g_num_sms = 0;
+
+}  // namespace
+
+int tc_num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0, n = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_num_sms = n > 0 ? n : 148;
+    }
+    return g_num_sms;
+}
+
+static void fill_params(TcParams& P, const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+                        const DeviceRouting& r, int* err, unsigned spin) {
+    memset(&P, 0, sizeof(P));
+    for (int i = 0; i < nmaps && i < kMaxMaps; ++i) P.maps[i] = maps[i];
+    for (int i = 0; i < nprob; ++i) P.prob[i] = probs[i];
+    P.nprob = nprob;
+    P.nmaps = nmaps < kMaxMaps ? nmaps : kMaxMaps;
+    P.r = r;
+    P.err = err;
+    P.spin = spin;
+}
+
+// Dense tile counts (host side) and a grid no larger than the work.
+template <int BN, bool kSwap>
+static int dense_tile_count(const GemmProblem& pr) {
+    using S = Shape<BN, kSwap>;
+    return ((pr.m_rows + S::kActRows - 1) / S::kActRows) * (pr.n / S::kOutCols);
+}
+
+cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
+                           const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    TcParams P;
+    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
+    const int sms = tc_num_sms();
+    int grid = sms;
+    if (!probs[0].grouped) {
+        long long tiles = 0;
+        for (int i = 0; i < nprob; ++i) {
+            P.dense_tiles[i] = bn == 256   ? dense_tile_count<256, false>(probs[i])
+                               : bn == 128 ? dense_tile_count<128, false>(probs[i])
+                                           : dense_tile_count<64, false>(probs[i]);
+            tiles += P.dense_tiles[i];
+        }
+        if (tiles < grid) grid = (int)tiles;
+        if (grid < 1) return cudaSuccess;
+    }
+    switch (bn) {
+        case 256: return launch_impl<256, 4, false>(P, grid, s);
+        case 128: return launch_impl<128, 6, false>(P, grid, s);
+        case 64: return launch_impl<64, 8, false>(P, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+                                  const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    TcParams P;
+    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
+    int grid = tc_num_sms();
+    if (!probs[0].grouped) {
+        long long tiles = 0;
+        for (int i = 0; i < nprob; ++i) {
+            P.dense_tiles[i] = dense_tile_count<kDecodeTN, true>(probs[i]);
+            tiles += P.dense_tiles[i];
+        }
+        if (tiles < grid) grid = (int)tiles;
+        if (grid < 1) return cudaSuccess;
+    }
+    return launch_impl<kDecodeTN, 10, true>(P, grid, s);
+}
+
+// ---------------------------------------------------------------- self-test
+__global__ void k_selftest_wait(int* err, unsigned spin) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, spin, err);  // nothing ever arrives
+}
+
+cudaError_t launch_selftest_wait(int* err, unsigned spin_limit, cudaStream_t s) {
+    k_selftest_wait<<<1, 32, 0, s>>>(err, spin_limit);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

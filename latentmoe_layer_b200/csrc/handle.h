@@ -1,0 +1,15 @@
+// handle.h -- host-side state of a LatentMoE layer handle.
+#pragma once
+#include "lmoe_internal.h"
+
+struct lmoe_handle {
+    lmoe_config cfg;
+    lmoe_weights w;
+    int* herr = nullptr;       // pinned, device-mapped error word (host view)
+    int* derr = nullptr;       // same word, device view
+    int gemm_path = 0;         // lmoe_option LMOE_OPT_GEMM_PATH
+    int fp64_all = 0;          // LMOE_OPT_ROUTER_FP64_ALL
+    float flag_delta = 4e-5f;  // LMOE_OPT_FLAG_DELTA
+    unsigned spin_limit = 1u << 24;
+    int num_sms = 148;
+};

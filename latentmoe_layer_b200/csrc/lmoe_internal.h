@@ -1,0 +1,99 @@
+// lmoe_internal.h -- structures shared by the host entry points and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/latentmoe.h"
+
+namespace lmoe {
+
+constexpr int kBM = 128;          // tensor-core tile rows (MMA M)
+constexpr int kBK = 64;           // K elements per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kSimtBM = 64;       // SIMT validation kernels tile rows
+constexpr int kDecodeTN = 32;     // token tile of the swap-AB decode variant (MMA N)
+constexpr float kBandEps = 1e-6f; // tie band of the routing rule
+constexpr int kMaxK = 64;
+constexpr int kMaxE = 1024;
+constexpr int kMaxG = 32;
+
+// Small block at the head of the workspace.
+struct WsStats {
+    int flagged;        // tokens appended to the fp64 re-check list
+    int distinct;       // experts with at least one token
+    int max_count;      // largest per-expert count
+    int device_error;   // lmoe_status from a device check
+    int pad[60];
+};
+
+// Epilogue kinds of the GEMM kernels.
+enum Epi : int {
+    EPI_F32 = 0,        // out fp32 = acc
+    EPI_BF16 = 1,       // out bf16 = acc
+    EPI_RELU2_BF16 = 2, // out bf16 = relu(acc)^2
+    EPI_SCALE_F32 = 3,  // out fp32 = row_scale[row] * acc
+    EPI_RELU2_F32 = 4,  // out fp32 = relu(acc)^2 (validation mode)
+};
+
+// One GEMM problem: out[m, n] = epi(sum_k A[m, k] B[n, k]) over up to two
+// K segments (segment 1 continues the same accumulator: K concatenation).
+// Dense problems have m_rows rows; grouped problems take their row ranges
+// from offsets[E+1] and B rows from expert e's block (b_rows_per_expert).
+struct GemmProblem {
+    int grouped;            // 0 dense, 1 grouped by expert
+    int m_rows;             // dense only
+    int n;                  // N (columns of out)
+    int nseg;               // 1 or 2
+    int kdim[2];            // K of each segment
+    int a_map[2], b_map[2]; // tensor-map indices (tensor-core path)
+    const void* a_ptr[2];   // operand pointers (SIMT path); A row stride = kdim[s]
+    const void* b_ptr[2];   // B row stride = kdim[s]
+    int b_rows_per_expert;  // grouped: rows of B per expert
+    int epi;
+    void* out;
+    long long ldo;          // elements
+    const float* row_scale; // EPI_SCALE_F32
+};
+
+struct DeviceRouting {
+    const int* offsets;     // [E+1] permuted row offset of each expert
+    const int* pfx128;      // [E+1] prefix of ceil(count/128)
+    const int* pfx64;       // [E+1] prefix of ceil(count/64)
+    const int* pfxdec;      // [E+1] prefix of ceil(count/kDecodeTN)
+    int E;
+};
+
+// Workspace carving for one call.
+struct Plan {
+    size_t total;
+    size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, blockcounts, perm,
+        slot, wperm, xbf, z, zperm, aperm, o, comb, as;
+    int T, A, nblk;
+};
+
+}  // namespace lmoe
+
+// ---- launchers (all asynchronous on `stream`; return cudaError_t) ----------
+struct lmoe_handle;
+namespace lmoe {
+cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStream_t s);
+cudaError_t launch_router_select(const lmoe_handle* h, const Plan& p, char* ws, bool fp64_all, cudaStream_t s);
+cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Plan& p, char* ws, bool all,
+                                   cudaStream_t s);
+cudaError_t launch_router_select64(const lmoe_handle* h, const Plan& p, char* ws, bool all, cudaStream_t s);
+cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_t* counts_out, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* offsets_E,
+                               int row_bytes, cudaStream_t s);
+cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
+                           cudaStream_t s);
+cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n,
+                                cudaStream_t s);
+cudaError_t launch_gemm_simt(const GemmProblem* probs, int nprob, bool a_f32, const DeviceRouting& r, int max_rows,
+                             cudaStream_t s);
+cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
+                           const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
+cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+                                  const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
+cudaError_t launch_selftest_wait(int* err, unsigned spin_limit, cudaStream_t s);
+int tc_num_sms();
+}  // namespace lmoe

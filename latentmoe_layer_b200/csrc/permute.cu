@@ -1,0 +1,258 @@
+// permute.cu -- token permutation, row gather, weighted combine and small
+// conversion kernels of the LatentMoE layer.
+//
+// The permutation is a deterministic counting sort of the (token, expert)
+// assignments by expert, stable in token id: permuted row
+//   offsets[e] + (number of earlier tokens routed to e)
+// holds token t's copy for expert e. It replaces the per-expert Python loop
+// over `expert_hit` with index_add_ ("Nemotron 3 Ultra 架构 QA", Q5.1, Q5.6):
+// expert e's rows are contiguous, so each expert's FFN is one GEMM over them,
+// and the combine sums each token's k rows in ascending expert id.
+#include <cuda_bf16.h>
+
+#include "handle.h"
+#include "lmoe_internal.h"
+#include "ptx.cuh"
+
+namespace lmoe {
+namespace {
+
+constexpr int kChunk = 256;  // tokens per counting block
+
+__global__ void k_count(const int32_t* __restrict__ idx, int T, int k, int E, int* __restrict__ blockcounts) {
+    extern __shared__ int hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
+    for (int i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x) atomicAdd(&hist[idx[i]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) blockcounts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// Inclusive block scan of 4 integer lanes at once (blockDim.x == 1024).
+__device__ void block_scan4(int4& v, int4* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int4 o;
+        o.x = __shfl_up_sync(0xFFFFFFFFu, v.x, off);
+        o.y = __shfl_up_sync(0xFFFFFFFFu, v.y, off);
+        o.z = __shfl_up_sync(0xFFFFFFFFu, v.z, off);
+        o.w = __shfl_up_sync(0xFFFFFFFFu, v.w, off);
+        if (lane >= off) {
+            v.x += o.x;
+            v.y += o.y;
+            v.z += o.z;
+            v.w += o.w;
+        }
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int4 t = warp_tot[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int4 o;
+            o.x = __shfl_up_sync(0xFFFFFFFFu, t.x, off);
+            o.y = __shfl_up_sync(0xFFFFFFFFu, t.y, off);
+            o.z = __shfl_up_sync(0xFFFFFFFFu, t.z, off);
+            o.w = __shfl_up_sync(0xFFFFFFFFu, t.w, off);
+            if (lane >= off) {
+                t.x += o.x;
+                t.y += o.y;
+                t.z += o.z;
+                t.w += o.w;
+            }
+        }
+        warp_tot[lane] = t;
+    }
+    __syncthreads();
+    if (warp > 0) {
+        int4 p = warp_tot[warp - 1];
+        v.x += p.x;
+        v.y += p.y;
+        v.z += p.z;
+        v.w += p.w;
+    }
+}
+
+__global__ void __launch_bounds__(1024)
+    k_scan(int* __restrict__ blockcounts, int nblk, int E, int* __restrict__ counts, int32_t* __restrict__ counts_out,
+           int* __restrict__ offsets, int* __restrict__ pfx128, int* __restrict__ pfx64, int* __restrict__ pfxdec,
+           WsStats* __restrict__ st) {
+    __shared__ int4 warp_tot[32];
+    __shared__ int red[2];
+    const int e = threadIdx.x;
+    int run = 0;
+    if (e < E) {
+        for (int b = 0; b < nblk; ++b) {
+            int v = blockcounts[(size_t)b * E + e];
+            blockcounts[(size_t)b * E + e] = run;
+            run += v;
+        }
+        counts[e] = run;
+        if (counts_out) counts_out[e] = run;
+    }
+    if (e < 2) red[e] = 0;
+    __syncthreads();
+    if (e < E && run > 0) {
+        atomicAdd(&red[0], 1);
+        atomicMax(&red[1], run);
+    }
+    int4 v = make_int4(run, (run + 127) / 128, (run + 63) / 64, (run + kDecodeTN - 1) / kDecodeTN);
+    int4 incl = v;
+    block_scan4(incl, warp_tot);
+    if (e < E) {
+        offsets[e] = incl.x - v.x;
+        pfx128[e] = incl.y - v.y;
+        pfx64[e] = incl.z - v.z;
+        pfxdec[e] = incl.w - v.w;
+        if (e == E - 1) {
+            offsets[E] = incl.x;
+            pfx128[E] = incl.y;
+            pfx64[E] = incl.z;
+            pfxdec[E] = incl.w;
+        }
+    }
+    __syncthreads();
+    if (e == 0) {
+        st->distinct = red[0];
+        st->max_count = red[1];
+    }
+}
+
+__global__ void k_scatter(const int32_t* __restrict__ idx, const float* __restrict__ w, int T, int k, int E,
+                          const int* __restrict__ blockcounts, const int* __restrict__ offsets, int* __restrict__ perm,
+                          int* __restrict__ slot, float* __restrict__ wperm) {
+    extern __shared__ int cursor[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        cursor[e] = offsets[e] + blockcounts[(size_t)blockIdx.x * E + e];
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
+    for (int t = t0; t < t1; ++t) {
+        for (int j = lane; j < k; j += 32) {
+            const int e = idx[(size_t)t * k + j];
+            const int pos = cursor[e];
+            cursor[e] = pos + 1;
+            perm[pos] = t;
+            slot[(size_t)t * k + j] = pos;
+            wperm[pos] = w[(size_t)t * k + j];
+        }
+        __syncwarp();
+    }
+}
+
+// dst[r, :] = src[perm[r], :] for r < offsets_E[0] (row_bytes multiple of 16).
+__global__ void k_gather(const uint4* __restrict__ src, uint4* __restrict__ dst, const int* __restrict__ perm,
+                         const int* __restrict__ total, int vec_per_row) {
+    const int rows = *total;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)rows * vec_per_row;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long r = i / vec_per_row, c = i % vec_per_row;
+        dst[i] = src[(long long)perm[r] * vec_per_row + c];
+    }
+}
+
+// comb[t, :] = sum_{j ascending} o[slot[t, j], :]   (o already carries w)
+template <bool kBf16>
+__global__ void __launch_bounds__(256)
+    k_combine(const float4* __restrict__ o, const int* __restrict__ slot, void* __restrict__ comb, int T, int k,
+              int L4) {
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        const int* sl = slot + (size_t)t * k;
+        for (int c = threadIdx.x; c < L4; c += blockDim.x) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < k; ++j) {
+                float4 v = __ldg(&o[(size_t)sl[j] * L4 + c]);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            if (kBf16) {
+                uint2 pk;
+                pk.x = pack_bf16x2(acc.x, acc.y);
+                pk.y = pack_bf16x2(acc.z, acc.w);
+                reinterpret_cast<uint2*>(comb)[(size_t)t * L4 + c] = pk;
+            } else {
+                reinterpret_cast<float4*>(comb)[(size_t)t * L4 + c] = acc;
+            }
+        }
+    }
+}
+
+__global__ void k_convert(const float4* __restrict__ x, uint2* __restrict__ xb, long long n4) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        float4 v = x[i];
+        xb[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
+}
+
+__global__ void k_copy_routing(const int* __restrict__ idx, const float* __restrict__ w, int32_t* __restrict__ io,
+                               float* __restrict__ wo, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        if (io) io[i] = idx[i];
+        if (wo) wo[i] = w[i];
+    }
+}
+
+inline int grid_cap(long long work, int per_block, int cap) {
+    long long g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    return (int)(g < cap ? g : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_t* counts_out, cudaStream_t s) {
+    const int E = h->cfg.num_experts, k = h->cfg.top_k;
+    int* bc = reinterpret_cast<int*>(ws + p.blockcounts);
+    const int32_t* idx = reinterpret_cast<const int32_t*>(ws + p.idx);
+    k_count<<<p.nblk, 256, E * sizeof(int), s>>>(idx, p.T, k, E, bc);
+    k_scan<<<1, 1024, 0, s>>>(bc, p.nblk, E, reinterpret_cast<int*>(ws + p.counts), counts_out,
+                              reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
+                              reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
+                              reinterpret_cast<WsStats*>(ws + p.stats));
+    k_scatter<<<p.nblk, 256, E * sizeof(int), s>>>(idx, reinterpret_cast<const float*>(ws + p.wgt), p.T, k, E, bc,
+                                                   reinterpret_cast<const int*>(ws + p.offsets),
+                                                   reinterpret_cast<int*>(ws + p.perm),
+                                                   reinterpret_cast<int*>(ws + p.slot),
+                                                   reinterpret_cast<float*>(ws + p.wperm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* total,
+                               int row_bytes, cudaStream_t s) {
+    const int vpr = row_bytes / 16;
+    int grid = grid_cap((long long)rows_total_max * vpr, 256, 148 * 16);
+    k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, total, vpr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
+                           cudaStream_t s) {
+    int grid = T < 148 * 8 ? T : 148 * 8;
+    if (out_bf16)
+        k_combine<true><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), slot, comb, T, k, L / 4);
+    else
+        k_combine<false><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), slot, comb, T, k, L / 4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStream_t s) {
+    long long n4 = n / 4;
+    k_convert<<<grid_cap(n4, 256, 148 * 16), 256, 0, s>>>(reinterpret_cast<const float4*>(x),
+                                                          reinterpret_cast<uint2*>(xb), n4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n,
+                                cudaStream_t s) {
+    if (!idx_out && !w_out) return cudaSuccess;
+    k_copy_routing<<<grid_cap(n, 256, 148 * 8), 256, 0, s>>>(idx, w, idx_out, w_out, n);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

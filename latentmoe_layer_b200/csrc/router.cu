@@ -1,0 +1,294 @@
+// router.cu -- routing kernels of the LatentMoE layer.
+//
+// Router ("Nemotron 3 Ultra 架构 QA", Q5.2/Q5.3; "Nemotron-3-Labs-Ultra-Math-SFT"
+// article, section 路由与共享专家): sigma = sigmoid(logits), choice = sigma +
+// e_score_correction_bias (selection only), grouped top-k with the 1e-6 tie
+// band in ascending id, weights = scale * sigma / sum(sigma of the selected).
+//
+// Two precisions of the same decision:
+//  * k_select<float, true>: from fp32 tensor-core logits. A token is flagged
+//    when any quantity that decides membership lies within a margin `delta`
+//    of a band edge; flagged tokens are appended to a list.
+//  * k_logits64 + k_select<double, false>: exact-product fp64 logits and the
+//    decision in fp64, for the flagged tokens (or for all tokens when x is fp32
+//    or in the fp32 validation mode).
+// With |fp32 choice - fp64 choice| <= delta/2 for every expert, unflagged
+// tokens provably get the fp64 decision: order statistics move by at most the
+// same bound, so every expert's distance to tau moves by at most delta and
+// every group score's distance to its tau by at most 2 delta.
+#include <float.h>
+#include <math.h>
+
+#include "handle.h"
+#include "lmoe_internal.h"
+
+namespace lmoe {
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ float sigmoid_t(float v) { return 1.0f / (1.0f + expf(-v)); }
+__device__ __forceinline__ double sigmoid_t(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+__device__ __forceinline__ unsigned first_n_bits(unsigned m, int n) {
+    unsigned r = 0;
+    for (int i = 0; i < n && m; ++i) {
+        unsigned low = m & (0u - m);
+        r |= low;
+        m ^= low;
+    }
+    return r;
+}
+
+// Warp-cooperative grouped top-k for one token. c[] and sig[] (length E) live
+// in this warp's shared memory. Writes idx (ascending) and weights; returns
+// true when the token must be re-decided in fp64 (kFlag only).
+template <typename F, bool kFlag>
+__device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int k, float scale, F delta,
+                            int32_t* idx_out, float* w_out) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    const F eps = (F)kBandEps;
+    const F ninf = -(F)INFINITY;
+    bool flag = false;
+    unsigned keep = 0xFFFFFFFFu;
+    const int per = E / G;
+    if (G > 1) {
+        F gs = ninf;
+        if (lane < G) {
+            F a = ninf, b = ninf;
+            for (int e = lane * per; e < (lane + 1) * per; ++e) {
+                F v = c[e];
+                if (v > a) {
+                    b = a;
+                    a = v;
+                } else if (v > b) {
+                    b = v;
+                }
+            }
+            gs = a + b;
+        }
+        int rank = 0;
+        for (int g = 0; g < G; ++g) {
+            F o = __shfl_sync(0xFFFFFFFFu, gs, g);
+            if (o > gs || (o == gs && g < lane)) ++rank;
+        }
+        unsigned kth = __ballot_sync(0xFFFFFFFFu, lane < G && rank == Gk - 1);
+        F tau = __shfl_sync(0xFFFFFFFFu, gs, __ffs(kth) - 1);
+        bool inA = lane < G && gs > tau + eps;
+        bool inB = lane < G && !inA && fabs(gs - tau) <= eps;
+        unsigned mA = __ballot_sync(0xFFFFFFFFu, inA);
+        unsigned mB = __ballot_sync(0xFFFFFFFFu, inB);
+        keep = mA | first_n_bits(mB, Gk - __popc(mA));
+        if (kFlag) {
+            F d = gs - tau;
+            bool near = lane < G && (fabs(d - eps) <= 2 * delta || fabs(d + eps) <= 2 * delta);
+            flag |= __any_sync(0xFFFFFFFFu, near);
+        }
+    }
+    // tau = k-th largest eligible choice score (k rounds of warp argmax).
+    const int nI = (E + 31) >> 5;
+    unsigned removed = 0;
+    F tau = ninf;
+    for (int j = 0; j < k; ++j) {
+        F best = ninf;
+        int be = 0x7FFFFFFF;
+        for (int i = 0; i < nI; ++i) {
+            int e = lane + (i << 5);
+            if (e < E && ((keep >> (e / per)) & 1u) && !((removed >> i) & 1u)) {
+                F v = c[e];
+                if (v > best) {
+                    best = v;
+                    be = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            F ob = __shfl_xor_sync(0xFFFFFFFFu, best, off);
+            int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+            if (ob > best || (ob == best && oe < be)) {
+                best = ob;
+                be = oe;
+            }
+        }
+        if (be != 0x7FFFFFFF && (be & 31) == lane) removed |= 1u << (be >> 5);
+        tau = best;
+    }
+    // A = {c > tau + eps}; the band |c - tau| <= eps fills the rest in ascending id.
+    int nA = 0;
+    for (int i = 0; i < nI; ++i) {
+        int e = lane + (i << 5);
+        bool inA = e < E && ((keep >> (e / per)) & 1u) && c[e] > tau + eps;
+        nA += __popc(__ballot_sync(0xFFFFFFFFu, inA));
+    }
+    const int need = k - nA;
+    int nout = 0, nband = 0;
+    bool near = false;
+    for (int i = 0; i < nI; ++i) {
+        int e = lane + (i << 5);
+        bool el = e < E && ((keep >> (e / per)) & 1u);
+        F v = el ? c[e] : (F)0;
+        bool inA = el && v > tau + eps;
+        bool inB = el && !inA && fabs(v - tau) <= eps;
+        unsigned mB = __ballot_sync(0xFFFFFFFFu, inB);
+        bool take = inA || (inB && nband + __popc(mB & lt) < need);
+        unsigned mT = __ballot_sync(0xFFFFFFFFu, take);
+        if (take) idx_out[nout + __popc(mT & lt)] = e;
+        nout += __popc(mT);
+        nband += __popc(mB);
+        if (kFlag && el) {
+            F d = v - tau;
+            near |= fabs(d - eps) <= delta || fabs(d + eps) <= delta;
+        }
+    }
+    if (kFlag) flag |= __any_sync(0xFFFFFFFFu, near);
+    __syncwarp();
+    // weights: scale * sigma_e / sum over the selected (fixed-order tree sum)
+    F part = 0;
+    for (int j = lane; j < k; j += 32) part += sig[idx_out[j]];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
+    for (int j = lane; j < k; j += 32) w_out[j] = (float)((F)scale * sig[idx_out[j]] / part);
+    return flag;
+}
+
+template <typename F, bool kFlag>
+__global__ void __launch_bounds__(kWarps * 32)
+    k_select(const F* __restrict__ logits, const float* __restrict__ bias, int T, int E, int G, int Gk, int k,
+             float scale, float delta, const int* __restrict__ list, const int* __restrict__ list_count,
+             int32_t* __restrict__ idx, float* __restrict__ wgt, int* __restrict__ flaglist,
+             int* __restrict__ flag_count) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    F* c = reinterpret_cast<F*>(smem_raw) + (size_t)warp * 2 * E;
+    F* sig = c + E;
+    const int n = list_count ? *list_count : T;
+    for (int item = blockIdx.x * kWarps + warp; item < n; item += gridDim.x * kWarps) {
+        const int t = list ? list[item] : item;
+        const F* lg = logits + (size_t)t * E;
+        for (int e = lane; e < E; e += 32) {
+            F s = sigmoid_t(lg[e]);
+            sig[e] = s;
+            c[e] = s + (F)bias[e];
+        }
+        __syncwarp();
+        bool flag = warp_select<F, kFlag>(c, sig, E, G, Gk, k, scale, (F)delta, idx + (size_t)t * k,
+                                          wgt + (size_t)t * k);
+        if (kFlag && flag && lane == 0) {
+            int pos = atomicAdd(flag_count, 1);
+            flaglist[pos] = t;
+        }
+        __syncwarp();
+    }
+}
+
+// fp64 logits: out[t, e] = sum_h x[t, h] * W_r[e, h]; the bf16 x bf16 (or
+// fp32 x bf16) products are exact in fp64. One work item = one token and a
+// chunk of 64 experts; the token's row is staged in shared memory as fp32.
+constexpr int kEChunk = 64;
+template <bool kXf32>
+__global__ void __launch_bounds__(256)
+    k_logits64(const void* __restrict__ x, const uint16_t* __restrict__ wr, int T, int E, int H,
+               const int* __restrict__ list, const int* __restrict__ list_count, double* __restrict__ out) {
+    extern __shared__ __align__(16) float xrow[];
+    const int n = list_count ? *list_count : T;
+    const int chunks = (E + kEChunk - 1) / kEChunk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (long long item = blockIdx.x; item < (long long)n * chunks; item += gridDim.x) {
+        const int li = (int)(item / chunks), ch = (int)(item % chunks);
+        const int t = list ? list[li] : li;
+        __syncthreads();
+        for (int h = threadIdx.x; h < H; h += blockDim.x) {
+            float v;
+            if (kXf32) {
+                v = static_cast<const float*>(x)[(size_t)t * H + h];
+            } else {
+                v = __uint_as_float((uint32_t) static_cast<const uint16_t*>(x)[(size_t)t * H + h] << 16);
+            }
+            xrow[h] = v;
+        }
+        __syncthreads();
+        for (int e = ch * kEChunk + warp; e < min(E, (ch + 1) * kEChunk); e += 8) {
+            const uint16_t* wrow = wr + (size_t)e * H;
+            double acc = 0.0;
+            for (int h = lane * 8; h < H; h += 256) {
+                uint4 pk = *reinterpret_cast<const uint4*>(wrow + h);
+                const uint32_t u[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fma((double)xrow[h + 2 * q], (double)__uint_as_float(u[q] << 16), acc);
+                    acc = fma((double)xrow[h + 2 * q + 1], (double)__uint_as_float(u[q] & 0xFFFF0000u), acc);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+            if (lane == 0) out[(size_t)t * E + e] = acc;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_select(const lmoe_handle* h, const Plan& p, char* ws, bool, cudaStream_t s) {
+    const lmoe_config& c = h->cfg;
+    int E = c.num_experts;
+    int blocks = (p.T + kWarps - 1) / kWarps;
+    if (blocks > 4 * h->num_sms) blocks = 4 * h->num_sms;
+    size_t smem = (size_t)kWarps * 2 * E * sizeof(float);
+    WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
+    k_select<float, true><<<blocks, kWarps * 32, smem, s>>>(
+        reinterpret_cast<const float*>(ws + p.logits), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
+        c.routed_scaling_factor, h->flag_delta, nullptr, nullptr, reinterpret_cast<int32_t*>(ws + p.idx),
+        reinterpret_cast<float*>(ws + p.wgt), reinterpret_cast<int*>(ws + p.flaglist), &st->flagged);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Plan& p, char* ws, bool all,
+                                   cudaStream_t s) {
+    const lmoe_config& c = h->cfg;
+    WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
+    const int* list = all ? nullptr : reinterpret_cast<const int*>(ws + p.flaglist);
+    const int* cnt = all ? nullptr : &st->flagged;
+    size_t smem = (size_t)c.hidden * sizeof(float);
+    int blocks = 2 * h->num_sms;
+    double* out = reinterpret_cast<double*>(ws + p.logits64);
+    if (smem > 48 * 1024) {
+        cudaError_t e = c.x_dtype == LMOE_FP32
+                            ? cudaFuncSetAttribute(k_logits64<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem)
+                            : cudaFuncSetAttribute(k_logits64<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    if (c.x_dtype == LMOE_FP32)
+        k_logits64<true><<<blocks, 256, smem, s>>>(x, static_cast<const uint16_t*>(h->w.router_w), p.T,
+                                                   c.num_experts, c.hidden, list, cnt, out);
+    else
+        k_logits64<false><<<blocks, 256, smem, s>>>(x, static_cast<const uint16_t*>(h->w.router_w), p.T,
+                                                    c.num_experts, c.hidden, list, cnt, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_select64(const lmoe_handle* h, const Plan& p, char* ws, bool all, cudaStream_t s) {
+    const lmoe_config& c = h->cfg;
+    WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
+    int E = c.num_experts;
+    size_t smem = (size_t)kWarps * 2 * E * sizeof(double);
+    if (smem > 48 * 1024) {
+        cudaError_t e =
+            cudaFuncSetAttribute(k_select<double, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int blocks = all ? (p.T + kWarps - 1) / kWarps : h->num_sms;
+    if (blocks > 4 * h->num_sms) blocks = 4 * h->num_sms;
+    if (blocks < 1) blocks = 1;
+    k_select<double, false><<<blocks, kWarps * 32, smem, s>>>(
+        reinterpret_cast<const double*>(ws + p.logits64), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
+        c.routed_scaling_factor, 0.f, all ? nullptr : reinterpret_cast<const int*>(ws + p.flaglist),
+        all ? nullptr : &st->flagged, reinterpret_cast<int32_t*>(ws + p.idx), reinterpret_cast<float*>(ws + p.wgt),
+        nullptr, nullptr);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -135,6 +135,25 @@ def host_tensor(w: LayerShape, key: str, seed: int = 0, rows=None) -> np.ndarray
     raise KeyError(key)
 
 
+def element(w: LayerShape, key: str, flat: int, seed: int = 0):
+    """Stored value of one element (uint16 bits for bf16, float for fp32), overrides included."""
+    for k, tid, shape, kind in tensor_specs(w):
+        if k != key:
+            continue
+        inner = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+        r, c = divmod(int(flat), inner)
+        if w.skew_hot and key == "x" and c == 0:
+            return 1.0 if w.x_f32 else BF16_ONE
+        if w.skew_hot and key == "router_w" and c == 0 and r < w.skew_hot:
+            return BF16_THREE
+        if kind == "b":
+            return float(uniform_f32(1, seed, tid, BIAS_LO, BIAS_HI, flat)[0])
+        if kind == "x" and w.x_f32:
+            return float(normal_f32(1, seed, tid, 1.0, flat)[0])
+        return int(normal_bf16(1, seed, tid, 1.0 if kind == "x" else W_SIGMA, flat)[0])
+    raise KeyError(key)
+
+
 def host_inputs(w: LayerShape, seed: int = 0) -> dict:
     return {k: host_tensor(w, k, seed) for k, _, _, _ in tensor_specs(w)}
 
@@ -173,4 +192,4 @@ def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
 
 __all__ = ["LayerShape", "WORKLOADS", "TINY", "NANO_DECODE", "ULTRA_DECODE", "ULTRA_PREFILL", "ULTRA_SKEW",
            "tensor_specs", "host_tensor", "host_inputs", "device_inputs", "build", "normal_bf16", "normal_f32",
-           "uniform_f32", "bf16_bits_to_f32", "TID_X", "TID_ROUTER"]
+           "uniform_f32", "bf16_bits_to_f32", "element", "TID_X", "TID_ROUTER"]

@@ -1,0 +1,135 @@
+"""The C ABI: exported symbols, argument validation and error paths."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import latentmoe_layer_b200 as lm
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    syms = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            txt = open(os.path.join(inc, f)).read()
+            syms |= set(re.findall(r"\b(latentmoe_\w+)\s*\(", txt))
+    return syms
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from latentmoe_layer_b200 import build
+    build.build()
+    return lm.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 9
+    out = subprocess.run(["nm", "-D", "--defined-only", lm.LIB_PATH], stdout=subprocess.PIPE, text=True).stdout
+    exported = set(re.findall(r"\bT (latentmoe_\w+)", out))
+    assert syms <= exported, syms - exported
+    for s in syms:
+        assert hasattr(lib, s)
+    assert set(lm.EXPORTS) <= syms
+
+
+def good_cfg(**kw):
+    w = synth.TINY
+    c = dict(hidden=w.H, latent=w.L, num_experts=w.E, top_k=w.k, n_group=w.G, topk_group=w.Gk,
+             expert_inter=w.I, shared_inter=w.Is, max_tokens=64, routed_scaling_factor=5.0, x_dtype=1, mode=0)
+    c.update(kw)
+    return lm.lmoe_config(**c)
+
+
+def fake_weights(addr=0x10000):
+    return lm.lmoe_weights(*([addr] * 8))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hidden=100), lm.LMOE_ERR_INVALID_ARG),          # not a multiple of 64
+    (dict(latent=0), lm.LMOE_ERR_INVALID_ARG),
+    (dict(top_k=0), lm.LMOE_ERR_INVALID_ARG),
+    (dict(top_k=17), lm.LMOE_ERR_INVALID_ARG),            # k > E
+    (dict(n_group=3), lm.LMOE_ERR_INVALID_ARG),           # E % G != 0
+    (dict(n_group=4, topk_group=5), lm.LMOE_ERR_INVALID_ARG),
+    (dict(n_group=4, topk_group=1, top_k=5), lm.LMOE_ERR_INVALID_ARG),  # k > kept experts
+    (dict(max_tokens=0), lm.LMOE_ERR_INVALID_ARG),
+    (dict(mode=7), lm.LMOE_ERR_INVALID_ARG),
+    (dict(x_dtype=3), lm.LMOE_ERR_INVALID_ARG),
+    (dict(routed_scaling_factor=float("nan")), lm.LMOE_ERR_INVALID_ARG),
+    (dict(num_experts=2048, top_k=2), lm.LMOE_ERR_UNSUPPORTED),
+    (dict(num_experts=64, n_group=64, topk_group=1, top_k=1), lm.LMOE_ERR_UNSUPPORTED),
+    (dict(num_experts=16, top_k=65), lm.LMOE_ERR_INVALID_ARG),
+])
+def test_invalid_configs_rejected_before_any_cuda_call(lib, kw, status):
+    s, h = lm.latentmoe_create(good_cfg(**kw), fake_weights())
+    assert s == status and not h.value
+
+
+def test_null_or_misaligned_weights_rejected(lib):
+    s, h = lm.latentmoe_create(good_cfg(), fake_weights(0))
+    assert s == lm.LMOE_ERR_INVALID_ARG and not h.value
+    s, h = lm.latentmoe_create(good_cfg(), fake_weights(0x10008))
+    assert s == lm.LMOE_ERR_INVALID_ARG and not h.value
+
+
+def test_null_handle_paths(lib):
+    assert lib.latentmoe_create(None, None, None) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_workspace_size(None, 4)[0] == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_forward(None, None, 1, None, None, 0, None) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_route(None, None, 1, None, None, None, None, 0, None) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(None, 0, 0) == lm.LMOE_ERR_INVALID_ARG
+    lm.latentmoe_destroy(None)
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lm.status_string(s) and lm.status_string(s) != "unknown status"
+    assert lm.status_string(99) == "unknown status"
+
+
+# ---------------------------------------------------------------- GPU error paths
+@pytest.mark.gpu
+def test_call_errors_leave_outputs_untouched(lib):
+    import torch
+    import helpers as H
+    shape = synth.TINY
+    layer, dev = H.device_layer(shape, max_tokens=64)
+    T = shape.T
+    y = torch.full((T, shape.H), 7.0, device="cuda")
+    ws, n = layer.workspace(T)
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    f = lm.latentmoe_forward
+    assert f(layer.h, None, T, y.data_ptr(), ws.data_ptr(), n, st) == lm.LMOE_ERR_INVALID_ARG
+    assert f(layer.h, dev["x"].data_ptr(), 65, y.data_ptr(), ws.data_ptr(), n, st) == lm.LMOE_ERR_INVALID_ARG
+    assert f(layer.h, dev["x"].data_ptr(), -1, y.data_ptr(), ws.data_ptr(), n, st) == lm.LMOE_ERR_INVALID_ARG
+    assert f(layer.h, dev["x"].data_ptr(), T, y.data_ptr(), ws.data_ptr(), n - 1, st) == lm.LMOE_ERR_WORKSPACE
+    assert f(layer.h, dev["x"].data_ptr(), T, y.data_ptr(), ws.data_ptr() + 16, n, st) == lm.LMOE_ERR_WORKSPACE
+    assert f(layer.h, dev["x"].data_ptr(), T, y.data_ptr() + 4, ws.data_ptr(), n, st) == lm.LMOE_ERR_INVALID_ARG
+    assert f(layer.h, dev["x"].data_ptr() + 8, T, y.data_ptr(), ws.data_ptr(), n, st) == lm.LMOE_ERR_INVALID_ARG
+    assert f(layer.h, dev["x"].data_ptr(), 0, y.data_ptr(), 0, 0, st) == lm.LMOE_OK
+    torch.cuda.synchronize()
+    assert bool((y == 7.0).all())
+    assert lm.latentmoe_set_option(layer.h, 0, 9) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, 3, 0) == lm.LMOE_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_bounded_wait_times_out_and_context_survives(lib):
+    import torch
+    import helpers as H
+    layer, dev = H.device_layer(synth.TINY)
+    layer.set_option(lm.OPT_SPIN_LIMIT, 20000)
+    assert lm.latentmoe_selftest_bounded_wait(layer.h) == lm.LMOE_ERR_TIMEOUT
+    layer.set_option(lm.OPT_SPIN_LIMIT, 1 << 24)
+    y = layer.forward(dev["x"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all()
+    assert layer.stats().device_error == 0

@@ -1,0 +1,185 @@
+"""GPU parity of the CUDA layer against the fp64 oracle, through the C ABI.
+
+Routing (expert indices, counts) must be bit-exact; weights match to fp32
+rounding; y within max-abs 2e-2 and relative Frobenius 1e-2 in bf16 mode and
+1e-5 relative Frobenius in the fp32 validation mode.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+
+import synth
+from synth import LayerShape, TINY, NANO_DECODE, ULTRA_DECODE, ULTRA_PREFILL, ULTRA_SKEW
+import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
+
+# several tiles and ragged tails in every dimension the kernels tile
+RAGGED = LayerShape("ragged", T=333, H=512, L=256, E=64, k=6, G=4, Gk=2, I=384, Is=640)
+RAGGED_X32 = replace(RAGGED, name="ragged_x32", x_f32=True, T=97)
+
+
+def run_and_compare(shape, mode=0, path=GEMM_AUTO, full=True):
+    import torch
+    layer, dev = H.device_layer(shape, mode=mode)
+    if path != GEMM_AUTO:
+        layer.set_option(0, path)
+    T = shape.T
+    idx = torch.empty((T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, shape.k), dtype=torch.float32, device="cuda")
+    counts = torch.empty((shape.E,), dtype=torch.int32, device="cuda")
+    y = layer.forward(dev["x"], idx=idx, w=w, counts=counts)
+    torch.cuda.synchronize()
+    host = synth.host_inputs(shape)
+    yref, iref, wref = H.oracle_forward(shape, host["x"], host, fp32_mode=(mode == 1))
+    assert np.array_equal(idx.cpu().numpy(), iref)
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(iref.ravel(), minlength=shape.E))
+    np.testing.assert_allclose(w.cpu().numpy(), wref, rtol=2e-6, atol=1e-6)
+    yg = y.cpu().numpy()
+    if mode == 1:
+        return H.assert_fp32_close(yg, yref), layer
+    return H.assert_bf16_close(yg, yref), layer
+
+
+@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_SIMT])
+def test_tiny_bf16(path):
+    run_and_compare(TINY, mode=0, path=path)
+
+
+def test_tiny_fp32_validation_mode():
+    run_and_compare(TINY, mode=1)
+
+
+@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT])
+def test_ragged_bf16(path):
+    run_and_compare(RAGGED, mode=0, path=path)
+
+
+def test_ragged_fp32_x_bf16_mode():
+    run_and_compare(RAGGED_X32, mode=0, path=GEMM_PREFILL)
+
+
+def test_ragged_fp32_validation_mode():
+    run_and_compare(RAGGED, mode=1)
+
+
+@pytest.mark.parametrize("path", [GEMM_AUTO, GEMM_PREFILL])
+def test_nano_decode_full(path):
+    (ma, rf), layer = run_and_compare(NANO_DECODE, mode=0, path=path)
+    st = layer.stats()
+    assert st.device_error == 0
+    print("nano_decode path=%d max_abs=%.3g rel_fro=%.3g flagged=%d distinct=%d" %
+          (path, ma, rf, st.flagged_tokens, st.distinct_experts))
+
+
+def _sampled_parity(shape, rows, route_rows, path=GEMM_AUTO):
+    """Full-size workload: routing of route_rows tokens and y of `rows` tokens vs the oracle."""
+    import torch
+    layer, dev = H.device_layer(shape)
+    if path != GEMM_AUTO:
+        layer.set_option(0, path)
+    H.check_device_inputs_match_generator(shape, dev)
+    T = shape.T
+    idx = torch.empty((T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, shape.k), dtype=torch.float32, device="cuda")
+    counts = torch.empty((shape.E,), dtype=torch.int32, device="cuda")
+    y = layer.forward(dev["x"], idx=idx, w=w, counts=counts)
+    y2 = layer.forward(dev["x"])
+    torch.cuda.synchronize()
+    st = layer.stats()
+    assert st.device_error == 0
+    assert torch.equal(y, y2), "two runs differ"
+    gi, gw, gc = idx.cpu().numpy(), w.cpu().numpy(), counts.cpu().numpy()
+    # properties at full size
+    assert gc.sum() == T * shape.k and np.array_equal(gc, np.bincount(gi.ravel(), minlength=shape.E))
+    assert np.all(np.diff(gi, axis=1) > 0)
+    np.testing.assert_allclose(gw.sum(1), shape.s, rtol=1e-5)
+    # routing of sampled tokens, bit-exact
+    wts = H.host_weights_for(shape, dev, [])
+    xr = H.host_x(shape, dev, route_rows)
+    ri, rw = H.oracle_route(shape, xr, wts)
+    assert np.array_equal(gi[route_rows], ri)
+    np.testing.assert_allclose(gw[route_rows], rw, rtol=2e-6, atol=1e-6)
+    # y of sampled rows
+    experts = np.unique(gi[rows])
+    wts = H.host_weights_for(shape, dev, experts)
+    yref, iref, _ = H.oracle_forward(shape, H.host_x(shape, dev, rows), wts)
+    assert np.array_equal(iref, gi[rows])
+    ma, rf = H.assert_bf16_close(y.cpu().numpy()[rows], yref)
+    hot = float(gc[:16].sum()) / gc.sum()
+    print("%s max_abs=%.3g rel_fro=%.3g flagged=%d distinct=%d max_count=%d hot16_share=%.3f" %
+          (shape.name, ma, rf, st.flagged_tokens, st.distinct_experts, st.max_expert_tokens, hot))
+    return layer
+
+
+def test_ultra_decode_sampled():
+    rng = np.random.default_rng(7)
+    _sampled_parity(ULTRA_DECODE, rows=np.sort(rng.choice(64, 6, replace=False)), route_rows=np.arange(64))
+
+
+def test_ultra_decode_prefill_tiles():
+    rng = np.random.default_rng(8)
+    _sampled_parity(ULTRA_DECODE, rows=np.sort(rng.choice(64, 3, replace=False)), route_rows=np.arange(64),
+                    path=GEMM_PREFILL)
+
+
+def test_ultra_prefill_sampled():
+    rng = np.random.default_rng(9)
+    T = ULTRA_PREFILL.T
+    rows = np.concatenate([[0, T - 1], rng.choice(T, 4, replace=False)])
+    _sampled_parity(ULTRA_PREFILL, rows=np.sort(rows), route_rows=np.sort(rng.choice(T, 256, replace=False)))
+
+
+def test_ultra_skew_sampled():
+    rng = np.random.default_rng(10)
+    T = ULTRA_SKEW.T
+    _sampled_parity(ULTRA_SKEW, rows=np.sort(rng.choice(T, 4, replace=False)),
+                    route_rows=np.sort(rng.choice(T, 256, replace=False)))
+
+
+def test_token_permutation_equivariance_bitwise():
+    import torch
+    layer, dev = H.device_layer(RAGGED)
+    layer.set_option(0, GEMM_PREFILL)
+    perm = torch.randperm(RAGGED.T, generator=torch.Generator().manual_seed(3)).cuda()
+    y = layer.forward(dev["x"]).clone()
+    yp = layer.forward(dev["x"][perm].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(yp, y[perm])
+
+
+def test_route_entry_point_matches_forward():
+    import torch
+    layer, dev = H.device_layer(RAGGED)
+    idx, w, counts = layer.route(dev["x"])
+    idx2 = torch.empty_like(idx)
+    w2 = torch.empty_like(w)
+    layer.forward(dev["x"], idx=idx2, w=w2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    assert int(counts.sum()) == RAGGED.T * RAGGED.k
+
+
+def test_zero_margin_shows_fp32_edge_cases_are_rechecked():
+    """With the near-edge margin forced to 0 no token is re-checked in fp64; the
+    default margin re-checks a few and routing is then exact on every token."""
+    import torch
+    shape = replace(ULTRA_DECODE, name="ultra_1k", T=1024)
+    layer, dev = H.device_layer(shape)
+    idx, _, _ = layer.route(dev["x"])
+    torch.cuda.synchronize()
+    st = layer.stats()
+    host = H.host_weights_for(shape, dev, [])
+    ri, _ = H.oracle_route(shape, H.host_x(shape, dev, np.arange(shape.T)), host)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    layer.set_option(2, 0)
+    idx0, _, _ = layer.route(dev["x"])
+    torch.cuda.synchronize()
+    st0 = layer.stats()
+    mism = int((idx0.cpu().numpy() != ri).any(1).sum())
+    print("flagged(default)=%d flagged(0)=%d mismatching tokens without re-check=%d" %
+          (st.flagged_tokens, st0.flagged_tokens, mism))
+    assert st0.flagged_tokens == 0 and st.flagged_tokens > 0
