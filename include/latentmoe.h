@@ -131,10 +131,19 @@ typedef struct {
     int distinct_experts;   /* experts with at least one token                  */
     int max_expert_tokens;  /* largest per-expert token count                   */
     int device_error;       /* lmoe_status recorded by a device-side check      */
+    int kernel_launches;    /* kernels the last route/forward call on the handle launched */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */
 lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out);
+
+/* Stage markers for timing inside a real call: when set (n >= 8), the next
+ * latentmoe_forward calls record events[i] (cudaEvent_t) on their stream at
+ * stage boundary i: 0 start, 1 routing done (router GEMM, selection, fp64
+ * re-check, permutation), 2 input GEMM (fc1 + shared up) done, 3 gather done,
+ * 4 expert up GEMM done, 5 expert down GEMM done, 6 combine done, 7 output
+ * GEMM done. NULL turns it off. The events are borrowed. */
+lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n);
 
 /* Runs one kernel that waits, with the handle's spin limit, on an mbarrier
  * that nothing ever completes, and returns the status it reports

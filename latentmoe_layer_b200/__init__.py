@@ -26,7 +26,7 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
-           "latentmoe_selftest_bounded_wait"]
+           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -43,7 +43,8 @@ class lmoe_weights(ctypes.Structure):
 
 class lmoe_stats(ctypes.Structure):
     _fields_ = [("flagged_tokens", ctypes.c_int), ("distinct_experts", ctypes.c_int),
-                ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int)]
+                ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int),
+                ("kernel_launches", ctypes.c_int)]
 
 
 class LmoeError(RuntimeError):
@@ -76,8 +77,10 @@ def load():
     lib.latentmoe_set_option.argtypes = [vp, i32, ctypes.c_longlong]
     lib.latentmoe_read_stats.argtypes = [vp, vp, ctypes.POINTER(lmoe_stats)]
     lib.latentmoe_selftest_bounded_wait.argtypes = [vp]
+    lib.latentmoe_set_profile_events.argtypes = [vp, vp, i32]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
-              "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait"):
+              "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
+              "latentmoe_set_profile_events"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -124,6 +127,10 @@ def latentmoe_read_stats(h, ws):
     st = lmoe_stats()
     s = load().latentmoe_read_stats(h, ws, ctypes.byref(st))
     return s, st
+
+
+def latentmoe_set_profile_events(h, events, n: int) -> int:
+    return load().latentmoe_set_profile_events(h, events, n)
 
 
 def latentmoe_selftest_bounded_wait(h) -> int:

@@ -132,8 +132,12 @@ lmoe_status check_weights(const lmoe_weights* w) {
 }
 
 // Tensor-core tile choice for a set of problem widths.
+#ifndef LMOE_MAX_BN
+#define LMOE_MAX_BN 256
+#endif
 int pick_bn(const int* ns, int cnt) {
     for (int bn : {256, 128, 64}) {
+        if (bn > LMOE_MAX_BN) continue;
         bool ok = true;
         for (int i = 0; i < cnt; ++i) ok = ok && ns[i] % bn == 0;
         if (ok) return bn;
@@ -204,6 +208,18 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
         if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
     } while (0)
 
+// Launch `expr`, which starts `n` kernels, and count them.
+#define LMOE_LAUNCH(n, expr)          \
+    do {                              \
+        LMOE_TRY(expr);               \
+        c.h->launches += (n);         \
+    } while (0)
+
+void mark(const Ctx& c, int i) {
+    if (c.h->prof_events && i < c.h->prof_n)
+        cudaEventRecord(static_cast<cudaEvent_t>(c.h->prof_events[i]), c.s);
+}
+
 __attribute__((unused)) lmoe_status take_device_error(lmoe_handle* h) {
     volatile int* he = h->herr;
     int v = *he;
@@ -240,17 +256,18 @@ lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int3
         Operand b[1][2] = {{{h->w.router_w, cf.num_experts}, {nullptr, 0}}};
         Ctx rc = c;
         rc.decode = c.decode && cf.num_experts % 128 == 0;
-        LMOE_TRY(run_gemm(rc, &pr, 1, a, b, false));
-        LMOE_TRY(launch_router_select(h, p, ws, false, c.s));
-        LMOE_TRY(launch_router_logits64(h, x, p, ws, false, c.s));
-        LMOE_TRY(launch_router_select64(h, p, ws, false, c.s));
+        LMOE_LAUNCH(1, run_gemm(rc, &pr, 1, a, b, false));
+        LMOE_LAUNCH(1, launch_router_select(h, p, ws, false, c.s));
+        LMOE_LAUNCH(1, launch_router_logits64(h, x, p, ws, false, c.s));
+        LMOE_LAUNCH(1, launch_router_select64(h, p, ws, false, c.s));
     } else {
-        LMOE_TRY(launch_router_logits64(h, x, p, ws, true, c.s));
-        LMOE_TRY(launch_router_select64(h, p, ws, true, c.s));
+        LMOE_LAUNCH(1, launch_router_logits64(h, x, p, ws, true, c.s));
+        LMOE_LAUNCH(1, launch_router_select64(h, p, ws, true, c.s));
     }
-    LMOE_TRY(launch_permute(h, p, ws, counts_out, c.s));
-    LMOE_TRY(launch_copy_routing(reinterpret_cast<const int*>(ws + p.idx), reinterpret_cast<const float*>(ws + p.wgt),
-                                 idx_out, w_out, (long long)p.T * cf.top_k, c.s));
+    LMOE_LAUNCH(3, launch_permute(h, p, ws, counts_out, c.s));
+    LMOE_LAUNCH((idx_out || w_out) ? 1 : 0,
+                launch_copy_routing(reinterpret_cast<const int*>(ws + p.idx), reinterpret_cast<const float*>(ws + p.wgt),
+                                    idx_out, w_out, (long long)p.T * cf.top_k, c.s));
     return LMOE_OK;
 }
 
@@ -328,9 +345,11 @@ lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_
     s = take_device_error(h);
     if (s != LMOE_OK) return s;
     Ctx c = make_ctx(h, p, ws, stream);
+    h->launches = 0;
     s = do_route(c, x, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
     return cuda_status(cudaGetLastError());
 }
 
@@ -348,8 +367,12 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
     const lmoe_config& cf = h->cfg;
     Ctx c = make_ctx(h, p, ws, stream);
     char* ws_c = c.ws;
+    h->launches = 0;
+    mark(c, 0);
     s = do_route(c, x, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
+    mark(c, 1);
+    const int gemm_kernels = c.simt ? 2 : 1;  // SIMT launches one kernel per problem
 
     const bool bf16 = cf.mode == LMOE_MODE_BF16;
     const int act = bf16 ? 2 : 4;
@@ -359,8 +382,8 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
     const void* xa = x;
     bool xa_f32 = cf.x_dtype == LMOE_FP32;
     if (bf16 && cf.x_dtype == LMOE_FP32) {
-        LMOE_TRY(launch_convert_x(static_cast<const float*>(x), reinterpret_cast<uint16_t*>(ws_c + p.xbf),
-                                  (long long)p.T * H, c.s));
+        LMOE_LAUNCH(1, launch_convert_x(static_cast<const float*>(x), reinterpret_cast<uint16_t*>(ws_c + p.xbf),
+                                        (long long)p.T * H, c.s));
         xa = ws_c + p.xbf;
         xa_f32 = false;
     }
@@ -379,11 +402,13 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
         pr[1].b_ptr[0] = h->w.shared_up_w;
         Operand a[2][2] = {{{xa, p.T}, {nullptr, 0}}, {{xa, p.T}, {nullptr, 0}}};
         Operand b[2][2] = {{{h->w.fc1_w, L}, {nullptr, 0}}, {{h->w.shared_up_w, Is}, {nullptr, 0}}};
-        LMOE_TRY(run_gemm(c, pr, 2, a, b, xa_f32));
+        LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
     }
+    mark(c, 2);
     // 6: expert-ordered copy of z
-    LMOE_TRY(launch_gather_rows(ws_c + p.z, ws_c + p.zperm, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
-                                reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
+    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, ws_c + p.zperm, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
+                                      reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
+    mark(c, 3);
     // 7: a = relu2(z_e W_up[e]^T)
     {
         GemmProblem pr = make_problem(1, 0, I, epi_relu2, ws_c + p.aperm, I);
@@ -393,8 +418,9 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
         pr.b_ptr[0] = h->w.up_w;
         Operand a[1][2] = {{{ws_c + p.zperm, A}, {nullptr, 0}}};
         Operand b[1][2] = {{{h->w.up_w, (long long)E * I}, {nullptr, 0}}};
-        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+        LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
     }
+    mark(c, 4);
     // 8: o = w * (a_e W_down[e]^T)
     {
         GemmProblem pr = make_problem(1, 0, L, EPI_SCALE_F32, ws_c + p.o, L);
@@ -405,11 +431,13 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
         pr.b_ptr[0] = h->w.down_w;
         Operand a[1][2] = {{{ws_c + p.aperm, A}, {nullptr, 0}}};
         Operand b[1][2] = {{{h->w.down_w, (long long)E * L}, {nullptr, 0}}};
-        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+        LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
     }
+    mark(c, 5);
     // 9: comb
-    LMOE_TRY(launch_combine(reinterpret_cast<const float*>(ws_c + p.o), reinterpret_cast<const int*>(ws_c + p.slot),
-                            ws_c + p.comb, p.T, cf.top_k, L, bf16, c.s));
+    LMOE_LAUNCH(1, launch_combine(reinterpret_cast<const float*>(ws_c + p.o), reinterpret_cast<const int*>(ws_c + p.slot),
+                                  ws_c + p.comb, p.T, cf.top_k, L, bf16, c.s));
+    mark(c, 6);
     // 10: y = comb W_fc2^T + a_s W_sd^T
     {
         GemmProblem pr = make_problem(0, p.T, H, EPI_F32, y, H);
@@ -422,9 +450,11 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
         pr.b_ptr[1] = h->w.shared_down_w;
         Operand a[1][2] = {{{ws_c + p.comb, p.T}, {ws_c + p.as, p.T}}};
         Operand b[1][2] = {{{h->w.fc2_w, H}, {h->w.shared_down_w, H}}};
-        LMOE_TRY(run_gemm(c, &pr, 1, a, b, !bf16));
+        LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
     }
+    mark(c, 7);
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
     return cuda_status(cudaGetLastError());
 }
 
@@ -477,6 +507,14 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
     out->distinct_experts = st.distinct;
     out->max_expert_tokens = st.max_count;
     out->device_error = st.device_error;
+    out->kernel_launches = h->launches;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n) {
+    if (!h || (events && n < 8)) return LMOE_ERR_INVALID_ARG;
+    h->prof_events = events;
+    h->prof_n = events ? n : 0;
     return LMOE_OK;
 }
 

@@ -10,11 +10,22 @@
 // Structure of one CTA (one per SM, persistent over tiles):
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles into a ring of
 //               shared-memory stages (mbarrier complete_tx), no multicast.
-//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.cta_group::1.kind::f16
-//               128 x BN x 16 per instruction, fp32 accumulators in TMEM,
-//               double-buffered so the epilogue of tile i overlaps tile i+1.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, the fused
-//               activation (relu2), weight scaling or bf16 rounding, stores.
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.cta_group::1.kind::f16,
+//               128 x BN x 16 per instruction, fp32 accumulation in TMEM.
+//   warps 2..   epilogue (4 or 8 warps; two per TMEM lane quarter for wide
+//               tiles): tcgen05.ld, then the fused activation (relu2), row
+//               weight or bf16 rounding, and the stores.
+//
+// Accumulation precision. The tensor core's fp32 accumulation over long K
+// carries several times the error of round-to-nearest fp32, and that error
+// grows with the accumulator's magnitude. Every GEMM output of the layer is
+// rounded to bf16 before the next GEMM, so that error turns into flipped bf16
+// roundings of large activations (one bf16 ulp at 64 is 0.5). K is therefore
+// accumulated in chunks of 4 k-blocks (256) in a ring of TMEM buffers; the
+// epilogue adds each chunk into fp32 registers, in order, while the MMA warp
+// fills the next buffer. Partial sums stay small, so the tensor-core error
+// no longer scales with the output, at the price of reading TMEM once per
+// chunk instead of once per tile.
 //
 // Two tile shapes share the code:
 //   kSwap = false  MMA M = 128 activation rows, N = BN weight rows.
@@ -29,11 +40,20 @@
 #include "lmoe_internal.h"
 #include "ptx.cuh"
 
+#ifndef LMOE_CHUNK_KB
+#define LMOE_CHUNK_KB 4   // k-blocks (of 64) per TMEM accumulation chunk
+#endif
+#ifndef LMOE_PROMOTE_F64
+#define LMOE_PROMOTE_F64 0  // 1: chunk partials are added into fp64 registers
+#endif
+#ifndef LMOE_MAX_BN
+#define LMOE_MAX_BN 256
+#endif
+
 namespace lmoe {
 namespace {
 
 constexpr int kMaxMaps = 8;
-constexpr int kThreads = 192;
 constexpr int kGroupM = 16;
 
 struct alignas(64) TcParams {
@@ -64,7 +84,16 @@ struct Shape {
     static constexpr int kStageBytes = kXBytes + kYBytes;
     static constexpr int kActRows = kSwap ? BN : 128;   // activation rows per tile
     static constexpr int kOutCols = kSwap ? 128 : BN;   // output columns per tile
-    static constexpr uint32_t kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+    // K is accumulated in chunks of kChunkKB k-blocks in TMEM; each chunk is
+    // added into fp32 registers by the epilogue (see the file comment).
+    static constexpr int kChunkKB = LMOE_CHUNK_KB;
+    static constexpr int kBufs = (4 * BN <= 512) ? 4 : 512 / BN;     // TMEM chunk buffers
+    static constexpr int kCols = kBufs * BN;
+    static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
+                                        : kCols <= 256 ? 256 : 512;
+    static constexpr int kEpiWarps = BN >= 128 ? 8 : 4;  // two warps per TMEM lane quarter for wide tiles
+    static constexpr int kColsPerThread = BN / (kEpiWarps / 4);
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
 };
 
 __device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
@@ -133,50 +162,51 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
     return ti;
 }
 
-template <int BN, bool kSwap>
+// Epilogue of one tile from the thread's fp32 accumulators acc[CW], which
+// hold accumulator columns c0 .. c0+CW-1 of TMEM lane `lane_row`.
+template <int BN, bool kSwap, int CW>
 __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const TileInfo& ti, int lane_row, int c0,
-                                               const uint32_t (&r)[16]) {
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+                                               float (&acc)[CW]) {
     const int epi = pr.epi;
     if (epi == EPI_RELU2_BF16 || epi == EPI_RELU2_F32) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float a = fmaxf(v[i], 0.f);
-            v[i] = a * a;
+        for (int i = 0; i < CW; ++i) {
+            float a = fmaxf(acc[i], 0.f);
+            acc[i] = a * a;
         }
     }
     if (!kSwap) {
-        // thread owns activation row (row0 + lane_row), columns col0 + c0 .. +15
+        // thread owns activation row (row0 + lane_row), output columns col0 + c0 ..
         if (lane_row >= ti.rows) return;
         const long long row = ti.row0 + lane_row;
         if (epi == EPI_SCALE_F32) {
             const float s = __ldg(&pr.row_scale[row]);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= s;
+            for (int i = 0; i < CW; ++i) acc[i] *= s;
         }
         if (epi == EPI_BF16 || epi == EPI_RELU2_BF16) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) + row * pr.ldo + ti.col0 + c0);
-            dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                pack_bf16x2(v[6], v[7]));
-            dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                pack_bf16x2(v[14], v[15]));
+#pragma unroll
+            for (int q = 0; q < CW / 8; ++q)
+                dst[q] = make_uint4(pack_bf16x2(acc[8 * q], acc[8 * q + 1]), pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]),
+                                    pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]),
+                                    pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
         } else {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + row * pr.ldo + ti.col0 + c0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int q = 0; q < CW / 4; ++q)
+                dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
         }
     } else {
-        // thread owns output column (col0 + lane_row); columns of the
-        // accumulator are tokens row0 + c0 .. +15.
+        // thread owns output column (col0 + lane_row); accumulator columns are
+        // the tile's tokens row0 + c0 + i. Lanes write consecutive columns.
         const long long col = ti.col0 + lane_row;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < CW; ++i) {
             const int tok = c0 + i;
             if (tok < ti.rows) {
                 const long long row = ti.row0 + tok;
-                float x = v[i];
+                float x = acc[i];
                 if (epi == EPI_SCALE_F32) x *= __ldg(&pr.row_scale[row]);
                 if (epi == EPI_BF16 || epi == EPI_RELU2_BF16)
                     static_cast<__nv_bfloat16*>(pr.out)[row * pr.ldo + col] = __float2bfloat16_rn(x);
@@ -187,9 +217,16 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
     }
 }
 
+__device__ __forceinline__ int tile_kblocks(const GemmProblem& pr) {
+    int n = pr.kdim[0] / kBK;
+    if (pr.nseg > 1) n += pr.kdim[1] / kBK;
+    return n;
+}
+
 template <int BN, int STAGES, bool kSwap>
-__global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
     using S = Shape<BN, kSwap>;
+    constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
@@ -197,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     uint8_t* sY = smem + STAGES * S::kXBytes;            // STAGES x kYBytes
     uint64_t* full = reinterpret_cast<uint64_t*>(sY + STAGES * S::kYBytes);
     uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* done = tempty + 2;
+    uint64_t* cfull = empty + STAGES;   // chunk accumulator ready (MMA -> epilogue)
+    uint64_t* cempty = cfull + NB;      // chunk accumulator drained (epilogue -> MMA)
+    uint64_t* done = cempty + NB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -208,9 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&cfull[b], 1);
+            mbar_init(&cempty[b], S::kEpiWarps);
         }
         mbar_init(done, 1);
         fence_mbar_init();
@@ -268,19 +305,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-        int stage = 0, acc = 0;
-        uint32_t phase = 0, acc_phase = 0;
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
-            const GemmProblem& pr = P.prob[ti.p];
-            if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, P.spin, err)) break;
-            tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)(acc * BN);
-            uint32_t accumulate = 0;
-            for (int sg = 0; sg < pr.nseg && ok; ++sg) {
-                const int kb_n = pr.kdim[sg] / kBK;
-                for (int kb = 0; kb < kb_n; ++kb) {
+            const int kb_total = tile_kblocks(P.prob[ti.p]);
+            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += CK) {
+                // next chunk accumulator must have been drained by the epilogue
+                if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, P.spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+                const int kb1 = min(kb_total, kb0 + CK);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
                         ok = false;
                         break;
@@ -291,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // +32 bytes per K step of 16 bf16 inside the 128-byte swizzled row
-                        umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, accumulate);
-                        accumulate = 1;
+                        umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                                  (kb > kb0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -300,12 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
                         phase ^= 1u;
                     }
                 }
-            }
-            if (!ok) break;
-            umma_commit(&tfull[acc]);
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
+                if (!ok) break;
+                umma_commit(&cfull[buf]);
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
             }
         }
         // all MMAs issued by this thread have completed before TMEM is freed
@@ -313,29 +353,70 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         mbar_wait_bounded(done, 0, 1u << 26, err);
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int ew = warp - 2;
+        const int q = warp & 3;                // TMEM lane quarter this warp may access
+        const int c0 = (ew >> 2) * CW;         // accumulator columns this warp owns
         const int lane_row = q * 32 + lane;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
             const GemmProblem& pr = P.prob[ti.p];
-            if (!mbar_wait_bounded(&tfull[acc], acc_phase, P.spin, err)) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(taddr + (uint32_t)c0, r);
-                tmem_ld_wait();
-                epilogue_store<BN, kSwap>(pr, ti, lane_row, c0, r);
+            const int kb_total = tile_kblocks(pr);
+#if LMOE_PROMOTE_F64
+            double accd[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) accd[i] = 0.0;
+#else
+            float acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = 0.f;
+#endif
+            for (int kb0 = 0; kb0 < kb_total; kb0 += CK) {
+                if (!mbar_wait_bounded(&cfull[buf], bphase, P.spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0);
+#pragma unroll
+                for (int c = 0; c < CW; c += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(taddr + (uint32_t)c, r0);
+                    if (c + 16 < CW) tmem_ld16(taddr + (uint32_t)(c + 16), r1);
+                    tmem_ld_wait();
+#if LMOE_PROMOTE_F64
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) accd[c + i] += (double)__uint_as_float(r0[i]);
+                    if (c + 16 < CW) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) accd[c + 16 + i] += (double)__uint_as_float(r1[i]);
+                    }
+#else
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[c + i] += __uint_as_float(r0[i]);
+                    if (c + 16 < CW) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[c + 16 + i] += __uint_as_float(r1[i]);
+                    }
+#endif
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cempty[buf]);
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
+            if (!ok) break;
+#if LMOE_PROMOTE_F64
+            float acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = (float)accd[i];
+#endif
+            epilogue_store<BN, kSwap, CW>(pr, ti, lane_row, c0, acc);
         }
     }
     __syncthreads();
@@ -354,10 +435,11 @@ template <int BN, int STAGES, bool kSwap>
 cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
     constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
     static_assert(smem <= 232448, "shared memory");
+    static_assert((2 * STAGES + 2 * Shape<BN, kSwap>::kBufs + 1) * 8 + 4 <= 256, "barrier area");
     cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    k_gemm_tc<BN, STAGES, kSwap><<<grid, kThreads, smem, s>>>(P);
+    k_gemm_tc<BN, STAGES, kSwap><<<grid, Shape<BN, kSwap>::kThreads, smem, s>>>(P);
     return cudaGetLastError();
 }
 

@@ -12,4 +12,7 @@ struct lmoe_handle {
     float flag_delta = 4e-5f;  // LMOE_OPT_FLAG_DELTA
     unsigned spin_limit = 1u << 24;
     int num_sms = 148;
+    int launches = 0;                  // kernels launched by the last call
+    void* const* prof_events = nullptr;  // latentmoe_set_profile_events
+    int prof_n = 0;
 };

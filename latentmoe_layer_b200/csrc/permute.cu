@@ -121,26 +121,40 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
+// One block per chunk of kChunk tokens: the chunk's expert ids and weights are
+// staged in shared memory, then one warp walks the tokens in order (the k
+// experts of a token are distinct, so its lanes never share a cursor).
 __global__ void k_scatter(const int32_t* __restrict__ idx, const float* __restrict__ w, int T, int k, int E,
                           const int* __restrict__ blockcounts, const int* __restrict__ offsets, int* __restrict__ perm,
                           int* __restrict__ slot, float* __restrict__ wperm) {
-    extern __shared__ int cursor[];
+    extern __shared__ int sm[];
+    int* cursor = sm;            // [E]
+    int* sidx = sm + E;          // [kChunk * k]
+    const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
+    const int n = (t1 - t0) * k;
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         cursor[e] = offsets[e] + blockcounts[(size_t)blockIdx.x * E + e];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) sidx[i] = idx[(size_t)t0 * k + i];
     __syncthreads();
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
-    const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
-    for (int t = t0; t < t1; ++t) {
-        for (int j = lane; j < k; j += 32) {
-            const int e = idx[(size_t)t * k + j];
-            const int pos = cursor[e];
-            cursor[e] = pos + 1;
-            perm[pos] = t;
-            slot[(size_t)t * k + j] = pos;
-            wperm[pos] = w[(size_t)t * k + j];
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        for (int tl = 0; tl < t1 - t0; ++tl) {
+            for (int j = lane; j < k; j += 32) {
+                const int e = sidx[tl * k + j];
+                const int pos = cursor[e];
+                cursor[e] = pos + 1;
+                sidx[tl * k + j] = pos;  // slot, written back below
+            }
+            __syncwarp();
         }
-        __syncwarp();
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int pos = sidx[i];
+        const size_t g = (size_t)t0 * k + i;
+        slot[g] = pos;
+        perm[pos] = t0 + i / k;
+        wperm[pos] = w[g];
     }
 }
 
@@ -215,7 +229,12 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
                               reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
                               reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
                               reinterpret_cast<WsStats*>(ws + p.stats));
-    k_scatter<<<p.nblk, 256, E * sizeof(int), s>>>(idx, reinterpret_cast<const float*>(ws + p.wgt), p.T, k, E, bc,
+    const size_t scatter_smem = (size_t)(E + kChunk * k) * sizeof(int);
+    if (scatter_smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_scatter<<<p.nblk, 256, scatter_smem, s>>>(idx, reinterpret_cast<const float*>(ws + p.wgt), p.T, k, E, bc,
                                                    reinterpret_cast<const int*>(ws + p.offsets),
                                                    reinterpret_cast<int*>(ws + p.perm),
                                                    reinterpret_cast<int*>(ws + p.slot),

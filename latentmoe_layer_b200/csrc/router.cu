@@ -6,16 +6,19 @@
 // band in ascending id, weights = scale * sigma / sum(sigma of the selected).
 //
 // Two precisions of the same decision:
-//  * k_select<float, true>: from fp32 tensor-core logits. A token is flagged
-//    when any quantity that decides membership lies within a margin `delta`
-//    of a band edge; flagged tokens are appended to a list.
+//  * k_select<float, true>: from fp32 tensor-core logits. The band rule only
+//    departs from the plain top-k by value when the k-th and (k+1)-th
+//    eligible choice scores are within 1e-6 (or the Gk-th and (Gk+1)-th group
+//    scores are); the token is flagged when either gap is within a margin
+//    `delta` of 1e-6, and flagged tokens are appended to a list.
 //  * k_logits64 + k_select<double, false>: exact-product fp64 logits and the
 //    decision in fp64, for the flagged tokens (or for all tokens when x is fp32
 //    or in the fp32 validation mode).
-// With |fp32 choice - fp64 choice| <= delta/2 for every expert, unflagged
-// tokens provably get the fp64 decision: order statistics move by at most the
-// same bound, so every expert's distance to tau moves by at most delta and
-// every group score's distance to its tau by at most 2 delta.
+// If every fp32 choice score is within delta/2 of its fp64 value, an
+// unflagged token's expert gap exceeds 1e-6 in fp64 too, so both precisions
+// select the top-k by value, and that set is the same in both because the gap
+// exceeds the perturbation; group scores (sums of two) move by at most delta,
+// which the 2*delta group margin covers.
 #include <float.h>
 #include <math.h>
 
@@ -80,22 +83,28 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
         unsigned mA = __ballot_sync(0xFFFFFFFFu, inA);
         unsigned mB = __ballot_sync(0xFFFFFFFFu, inB);
         keep = mA | first_n_bits(mB, Gk - __popc(mA));
-        if (kFlag) {
-            F d = gs - tau;
-            bool near = lane < G && (fabs(d - eps) <= 2 * delta || fabs(d + eps) <= 2 * delta);
-            flag |= __any_sync(0xFFFFFFFFu, near);
+        if (kFlag && Gk < G) {
+            unsigned nxt = __ballot_sync(0xFFFFFFFFu, lane < G && rank == Gk);
+            F below = __shfl_sync(0xFFFFFFFFu, gs, __ffs(nxt) - 1);
+            flag |= (tau - below) <= eps + 2 * delta;
         }
     }
-    // tau = k-th largest eligible choice score (k rounds of warp argmax).
+    // eligibility of this lane's experts e = lane + 32 i, one bit per i
     const int nI = (E + 31) >> 5;
+    unsigned elig = 0;
+    for (int i = 0; i < nI; ++i) {
+        const int e = lane + (i << 5);
+        if (e < E && ((keep >> (e / per)) & 1u)) elig |= 1u << i;
+    }
+    // tau = k-th largest eligible choice score (k rounds of warp argmax).
     unsigned removed = 0;
-    F tau = ninf;
-    for (int j = 0; j < k; ++j) {
+    F tau = ninf, next = ninf;
+    for (int j = 0; j < (kFlag ? k + 1 : k); ++j) {
         F best = ninf;
         int be = 0x7FFFFFFF;
         for (int i = 0; i < nI; ++i) {
-            int e = lane + (i << 5);
-            if (e < E && ((keep >> (e / per)) & 1u) && !((removed >> i) & 1u)) {
+            const int e = lane + (i << 5);
+            if (((elig & ~removed) >> i) & 1u) {
                 F v = c[e];
                 if (v > best) {
                     best = v;
@@ -113,21 +122,22 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
             }
         }
         if (be != 0x7FFFFFFF && (be & 31) == lane) removed |= 1u << (be >> 5);
-        tau = best;
+        if (j < k) tau = best;
+        else next = best;  // (k+1)-th largest eligible score, -inf if there is none
     }
+    if (kFlag) flag |= (tau - next) <= eps + delta;
     // A = {c > tau + eps}; the band |c - tau| <= eps fills the rest in ascending id.
     int nA = 0;
     for (int i = 0; i < nI; ++i) {
-        int e = lane + (i << 5);
-        bool inA = e < E && ((keep >> (e / per)) & 1u) && c[e] > tau + eps;
+        const int e = lane + (i << 5);
+        bool inA = ((elig >> i) & 1u) && c[e] > tau + eps;
         nA += __popc(__ballot_sync(0xFFFFFFFFu, inA));
     }
     const int need = k - nA;
     int nout = 0, nband = 0;
-    bool near = false;
     for (int i = 0; i < nI; ++i) {
-        int e = lane + (i << 5);
-        bool el = e < E && ((keep >> (e / per)) & 1u);
+        const int e = lane + (i << 5);
+        const bool el = (elig >> i) & 1u;
         F v = el ? c[e] : (F)0;
         bool inA = el && v > tau + eps;
         bool inB = el && !inA && fabs(v - tau) <= eps;
@@ -137,12 +147,7 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
         if (take) idx_out[nout + __popc(mT & lt)] = e;
         nout += __popc(mT);
         nband += __popc(mB);
-        if (kFlag && el) {
-            F d = v - tau;
-            near |= fabs(d - eps) <= delta || fabs(d + eps) <= delta;
-        }
     }
-    if (kFlag) flag |= __any_sync(0xFFFFFFFFu, near);
     __syncwarp();
     // weights: scale * sigma_e / sum over the selected (fixed-order tree sum)
     F part = 0;
@@ -185,40 +190,47 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // fp64 logits: out[t, e] = sum_h x[t, h] * W_r[e, h]; the bf16 x bf16 (or
 // fp32 x bf16) products are exact in fp64. One work item = one token and a
-// chunk of 64 experts; the token's row is staged in shared memory as fp32.
+// chunk of 64 experts; the token's row is staged in shared memory as fp64 and
+// read as 16-byte vectors (conflict-free), each lane covering 8 consecutive h.
 constexpr int kEChunk = 64;
 template <bool kXf32>
 __global__ void __launch_bounds__(256)
     k_logits64(const void* __restrict__ x, const uint16_t* __restrict__ wr, int T, int E, int H,
                const int* __restrict__ list, const int* __restrict__ list_count, double* __restrict__ out) {
-    extern __shared__ __align__(16) float xrow[];
+    extern __shared__ __align__(16) double xrow[];
     const int n = list_count ? *list_count : T;
     const int chunks = (E + kEChunk - 1) / kEChunk;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int cur = -1;
     for (long long item = blockIdx.x; item < (long long)n * chunks; item += gridDim.x) {
         const int li = (int)(item / chunks), ch = (int)(item % chunks);
         const int t = list ? list[li] : li;
-        __syncthreads();
-        for (int h = threadIdx.x; h < H; h += blockDim.x) {
-            float v;
-            if (kXf32) {
-                v = static_cast<const float*>(x)[(size_t)t * H + h];
-            } else {
-                v = __uint_as_float((uint32_t) static_cast<const uint16_t*>(x)[(size_t)t * H + h] << 16);
+        if (t != cur) {
+            __syncthreads();
+            for (int h = threadIdx.x; h < H; h += blockDim.x) {
+                float v;
+                if (kXf32) {
+                    v = static_cast<const float*>(x)[(size_t)t * H + h];
+                } else {
+                    v = __uint_as_float((uint32_t) static_cast<const uint16_t*>(x)[(size_t)t * H + h] << 16);
+                }
+                xrow[h] = (double)v;
             }
-            xrow[h] = v;
+            __syncthreads();
+            cur = t;
         }
-        __syncthreads();
         for (int e = ch * kEChunk + warp; e < min(E, (ch + 1) * kEChunk); e += 8) {
             const uint16_t* wrow = wr + (size_t)e * H;
             double acc = 0.0;
             for (int h = lane * 8; h < H; h += 256) {
-                uint4 pk = *reinterpret_cast<const uint4*>(wrow + h);
+                const uint4 pk = *reinterpret_cast<const uint4*>(wrow + h);
+                const double2* xv = reinterpret_cast<const double2*>(xrow + h);
                 const uint32_t u[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    acc = fma((double)xrow[h + 2 * q], (double)__uint_as_float(u[q] << 16), acc);
-                    acc = fma((double)xrow[h + 2 * q + 1], (double)__uint_as_float(u[q] & 0xFFFF0000u), acc);
+                    const double2 xx = xv[q];
+                    acc = fma(xx.x, (double)__uint_as_float(u[q] << 16), acc);
+                    acc = fma(xx.y, (double)__uint_as_float(u[q] & 0xFFFF0000u), acc);
                 }
             }
 #pragma unroll
@@ -250,7 +262,7 @@ cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Pl
     WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
     const int* list = all ? nullptr : reinterpret_cast<const int*>(ws + p.flaglist);
     const int* cnt = all ? nullptr : &st->flagged;
-    size_t smem = (size_t)c.hidden * sizeof(float);
+    size_t smem = (size_t)c.hidden * sizeof(double);
     int blocks = 2 * h->num_sms;
     double* out = reinterpret_cast<double*>(ws + p.logits64);
     if (smem > 48 * 1024) {
