@@ -137,6 +137,28 @@ typedef struct {
  * for tests and benchmarks, not for the hot path). */
 lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out);
 
+/* Routing for callers that cannot allocate device memory (a real-time or
+ * latency-critical section where cudaMalloc's implicit synchronisation is not
+ * allowed, a runtime whose device memory belongs to a fixed arena, a plugin
+ * host that forbids allocation from extension code). Same outputs as
+ * latentmoe_route, but there is no workspace argument and the call allocates
+ * nothing: its scratch is an 8 MiB array in this library's static device
+ * memory, held by every GPU that loads the library until the process exits.
+ * The pages have no counterpart of this entry point.
+ *  - Capacity: routing needs about 6.5 KiB per token at E = 512, k = 22, so
+ *    T up to roughly 1200 tokens fits at the Ultra shape; a T whose scratch
+ *    need exceeds 8 MiB returns LMOE_ERR_WORKSPACE and launches nothing.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears what must start at zero. Calls whose GPU work
+ *    overlaps (other streams, other threads, other handles) race on it:
+ *    order them on one stream or synchronise between them.
+ * The handle comes from latentmoe_create as usual. */
+lmoe_status latentmoe_route_noalloc(lmoe_handle* h, const void* x, int T, int32_t* topk_idx, float* topk_w,
+                                    int32_t* expert_counts, void* stream);
+
 /* Stage markers for timing inside a real call: when set (n >= 8), the next
  * latentmoe_forward calls record events[i] (cudaEvent_t) on their stream at
  * stage boundary i: 0 start, 1 routing done (router GEMM, selection, fp64

@@ -26,7 +26,7 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
-           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events"]
+           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -78,9 +78,10 @@ def load():
     lib.latentmoe_read_stats.argtypes = [vp, vp, ctypes.POINTER(lmoe_stats)]
     lib.latentmoe_selftest_bounded_wait.argtypes = [vp]
     lib.latentmoe_set_profile_events.argtypes = [vp, vp, i32]
+    lib.latentmoe_route_noalloc.argtypes = [vp, vp, i32, vp, vp, vp, vp]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
-              "latentmoe_set_profile_events"):
+              "latentmoe_set_profile_events", "latentmoe_route_noalloc"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -131,6 +132,11 @@ def latentmoe_read_stats(h, ws):
 
 def latentmoe_set_profile_events(h, events, n: int) -> int:
     return load().latentmoe_set_profile_events(h, events, n)
+
+
+def latentmoe_route_noalloc(h, x, T, idx, w, counts, stream) -> int:
+    """Routing with the library's static scratch (no workspace, no allocation)."""
+    return load().latentmoe_route_noalloc(h, x, T, idx, w, counts, stream)
 
 
 def latentmoe_selftest_bounded_wait(h) -> int:

@@ -20,6 +20,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "handle.h"
@@ -533,3 +534,66 @@ lmoe_status latentmoe_selftest_bounded_wait(lmoe_handle* h) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Routing without any allocation.
+//
+// Some callers cannot allocate device memory at the moment they route: code
+// running inside a real-time or latency-critical section where cudaMalloc's
+// implicit synchronisation is not allowed, inference runtimes whose memory is
+// owned by a fixed arena, plugin hosts that forbid allocation from extension
+// code. latentmoe_route_noalloc gives them routing with no workspace argument:
+// its scratch is the file-scope array below, which every GPU that loads this
+// library holds until the process exits.
+static constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is asked from the
+// runtime once per device (with that device current) and cached.
+lmoe_status noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LMOE_ERR_CUDA;
+    if (dev >= kMaxDevices) return LMOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LMOE_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LMOE_OK;
+}
+}  // namespace
+
+extern "C" lmoe_status latentmoe_route_noalloc(lmoe_handle* h, const void* x, int T, int32_t* topk_idx,
+                                               float* topk_w, int32_t* expert_counts, void* stream) {
+    if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!x || !aligned(x, 16)) return LMOE_ERR_INVALID_ARG;
+    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+        (expert_counts && !aligned(expert_counts, 4)))
+        return LMOE_ERR_INVALID_ARG;
+    Plan p;
+    plan_of(h->cfg, T, p);
+    // routing touches only the buffers up to the row weights (they come first in the plan)
+    const size_t need = p.wperm + al256((size_t)p.A * 4);
+    if (need > kNoAllocScratchBytes) return LMOE_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    lmoe_status s = noalloc_scratch(&scratch);
+    if (s != LMOE_OK) return s;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    Ctx c = make_ctx(h, p, scratch, stream);
+    h->launches = 0;
+    s = do_route(c, x, topk_idx, topk_w, expert_counts);  // clears the stats block first
+    if (s != LMOE_OK) return s;
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
