@@ -47,16 +47,22 @@ bool get_encoder() {
     return true;
 }
 
-// bf16 row-major [rows, cols] with cols contiguous; box = 64 columns (one
-// 128-byte swizzle row) x box_rows rows.
-bool encode_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+// Row-major [rows, cols] (cols contiguous), 128-byte-swizzled boxes of
+// 128 bytes x box_rows rows.
+bool encode_2d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows, bool f32) {
+    const int esz = f32 ? 4 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * esz};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
-    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// bf16 operand tiles: 64 columns (one 128-byte swizzle row) x box_rows rows.
+bool encode_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+    return encode_2d(m, base, rows, cols, box_rows, false);
 }
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -184,6 +190,16 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
                 return cudaErrorInvalidValue;
             probs[i].b_map[sg] = nm++;
         }
+    // output maps for the bulk tensor stores of non-swapped tiles (32-row slabs)
+    for (int i = 0; i < nprob && !swap; ++i) {
+        const bool f32_out = probs[i].epi == EPI_F32 || probs[i].epi == EPI_SCALE_F32 || probs[i].epi == EPI_RELU2_F32;
+        const long long rows = probs[i].grouped ? (long long)c.p->A : probs[i].m_rows;
+        if (probs[i].ldo != probs[i].n || !encode_2d(&maps[nm], probs[i].out, rows, probs[i].n, 32, f32_out)) {
+            probs[i].out_map = -1;
+            continue;
+        }
+        probs[i].out_map = nm++;
+    }
     if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
     return launch_gemm_tc(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
 }
@@ -198,6 +214,7 @@ GemmProblem make_problem(int grouped, int m_rows, int n, int epi, void* out, lon
     p.epi = epi;
     p.out = out;
     p.ldo = ldo;
+    p.out_map = -1;
     return p;
 }
 

@@ -94,6 +94,8 @@ struct Shape {
     static constexpr int kEpiWarps = BN >= 128 ? 8 : 4;  // two warps per TMEM lane quarter for wide tiles
     static constexpr int kColsPerThread = BN / (kEpiWarps / 4);
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    // per epilogue warp: one 32-row x 128-byte output box, 128-byte swizzled, for bulk tensor stores
+    static constexpr int kStageOutBytes = kSwap ? 0 : 4096;
 };
 
 __device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
@@ -164,10 +166,16 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
 
 // Epilogue of one tile from the thread's fp32 accumulators acc[CW], which
 // hold accumulator columns c0 .. c0+CW-1 of TMEM lane `lane_row`.
+// Non-swapped tiles with an output tensor map are written with bulk tensor
+// stores: the warp stages its 32 rows x 128 bytes in shared memory with the
+// 128-byte swizzle (conflict-free writes) and one lane issues the store. Rows
+// past a dense problem's end are clipped by the tensor bounds; a grouped tile
+// whose 32-row slab runs into the next expert's rows uses plain masked stores.
 template <int BN, bool kSwap, int CW>
 __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const TileInfo& ti, int lane_row, int c0,
-                                               float (&acc)[CW]) {
+                                               float (&acc)[CW], const CUtensorMap* omap, uint8_t* stage) {
     const int epi = pr.epi;
+    const int lane = threadIdx.x & 31;
     if (epi == EPI_RELU2_BF16 || epi == EPI_RELU2_F32) {
 #pragma unroll
         for (int i = 0; i < CW; ++i) {
@@ -176,15 +184,55 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
         }
     }
     if (!kSwap) {
+        const bool bf16_out = epi == EPI_BF16 || epi == EPI_RELU2_BF16;
+        const int slab0 = lane_row - lane;  // first row of this warp's 32-row slab
+        if (omap && (!pr.grouped || slab0 + 32 <= ti.rows)) {
+            if (epi == EPI_SCALE_F32) {
+                const float sc = __ldg(&pr.row_scale[ti.row0 + lane_row]);
+#pragma unroll
+                for (int i = 0; i < CW; ++i) acc[i] *= sc;
+            }
+            uint8_t* myrow = stage + lane * 128;
+            constexpr int kGroupsF32 = CW / 32, kGroupsBf16 = CW / 64;
+            const int ngroups = bf16_out ? kGroupsBf16 : kGroupsF32;
+#pragma unroll
+            for (int g = 0; g < (CW / 32); ++g) {
+                if (g >= ngroups) break;
+                if (lane == 0) bulk_wait_read_all();  // staging buffer free again
+                __syncwarp();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v;
+                    if (bf16_out) {
+                        const int b = g * 64 + c * 8;
+                        v = make_uint4(pack_bf16x2(acc[b], acc[b + 1]), pack_bf16x2(acc[b + 2], acc[b + 3]),
+                                       pack_bf16x2(acc[b + 4], acc[b + 5]), pack_bf16x2(acc[b + 6], acc[b + 7]));
+                    } else {
+                        const int b = g * 32 + c * 4;
+                        v = make_uint4(__float_as_uint(acc[b]), __float_as_uint(acc[b + 1]),
+                                       __float_as_uint(acc[b + 2]), __float_as_uint(acc[b + 3]));
+                    }
+                    *reinterpret_cast<uint4*>(myrow + ((c ^ (lane & 7)) << 4)) = v;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = ti.col0 + c0 + g * (bf16_out ? 64 : 32);
+                    tma_store_2d(omap, stage, x, ti.row0 + slab0);
+                    bulk_commit();
+                }
+            }
+            return;
+        }
         // thread owns activation row (row0 + lane_row), output columns col0 + c0 ..
         if (lane_row >= ti.rows) return;
         const long long row = ti.row0 + lane_row;
         if (epi == EPI_SCALE_F32) {
-            const float s = __ldg(&pr.row_scale[row]);
+            const float sc = __ldg(&pr.row_scale[row]);
 #pragma unroll
-            for (int i = 0; i < CW; ++i) acc[i] *= s;
+            for (int i = 0; i < CW; ++i) acc[i] *= sc;
         }
-        if (epi == EPI_BF16 || epi == EPI_RELU2_BF16) {
+        if (bf16_out) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) + row * pr.ldo + ti.col0 + c0);
 #pragma unroll
             for (int q = 0; q < CW / 8; ++q)
@@ -232,7 +280,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
     uint8_t* sX = smem;                                  // STAGES x kXBytes
     uint8_t* sY = smem + STAGES * S::kXBytes;            // STAGES x kYBytes
-    uint64_t* full = reinterpret_cast<uint64_t*>(sY + STAGES * S::kYBytes);
+    uint8_t* sOut = sY + STAGES * S::kYBytes;            // kEpiWarps x kStageOutBytes
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + S::kEpiWarps * S::kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* cfull = empty + STAGES;   // chunk accumulator ready (MMA -> epilogue)
     uint64_t* cempty = cfull + NB;      // chunk accumulator drained (epilogue -> MMA)
@@ -416,8 +465,10 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
 #pragma unroll
             for (int i = 0; i < CW; ++i) acc[i] = (float)accd[i];
 #endif
-            epilogue_store<BN, kSwap, CW>(pr, ti, lane_row, c0, acc);
+            const CUtensorMap* omap = pr.out_map >= 0 ? &P.maps[pr.out_map] : nullptr;
+            epilogue_store<BN, kSwap, CW>(pr, ti, lane_row, c0, acc, omap, sOut + ew * S::kStageOutBytes);
         }
+        if (!kSwap && lane == 0) bulk_wait_all();  // this warp's bulk stores are complete
     }
     __syncthreads();
     if (warp == 1) {
@@ -428,7 +479,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
 
 template <int BN, int STAGES, bool kSwap>
 constexpr size_t smem_bytes() {
-    return 1024 + (size_t)STAGES * Shape<BN, kSwap>::kStageBytes + 256;
+    using S = Shape<BN, kSwap>;
+    return 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 256;
 }
 
 template <int BN, int STAGES, bool kSwap>

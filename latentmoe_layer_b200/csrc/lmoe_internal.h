@@ -53,6 +53,7 @@ struct GemmProblem {
     void* out;
     long long ldo;          // elements
     const float* row_scale; // EPI_SCALE_F32
+    int out_map;            // tensor map of `out` for bulk tensor stores (-1: plain stores)
 };
 
 struct DeviceRouting {

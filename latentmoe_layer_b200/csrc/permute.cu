@@ -85,10 +85,15 @@ __global__ void __launch_bounds__(1024)
     const int e = threadIdx.x;
     int run = 0;
     if (e < E) {
-        for (int b = 0; b < nblk; ++b) {
-            int v = blockcounts[(size_t)b * E + e];
-            blockcounts[(size_t)b * E + e] = run;
-            run += v;
+        for (int b0 = 0; b0 < nblk; b0 += 8) {  // 8 independent loads in flight
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = b0 + j < nblk ? blockcounts[(size_t)(b0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (b0 + j < nblk) blockcounts[(size_t)(b0 + j) * E + e] = run;
+                run += v[j];
+            }
         }
         counts[e] = run;
         if (counts_out) counts_out[e] = run;
@@ -121,32 +126,48 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
-// One block per chunk of kChunk tokens: the chunk's expert ids and weights are
-// staged in shared memory, then one warp walks the tokens in order (the k
-// experts of a token are distinct, so its lanes never share a cursor).
-__global__ void k_scatter(const int32_t* __restrict__ idx, const float* __restrict__ w, int T, int k, int E,
-                          const int* __restrict__ blockcounts, const int* __restrict__ offsets, int* __restrict__ perm,
-                          int* __restrict__ slot, float* __restrict__ wperm) {
+// One block per chunk of kChunk tokens, 8 warps of 32 tokens each. The
+// chunk's expert ids are staged in shared memory; each warp counts its tokens
+// per expert, a prefix over the warps gives each warp its start inside every
+// expert's range, then each warp walks its 32 tokens in order (the k experts
+// of a token are distinct, so its lanes never share a cursor). The result is
+// the order of token id within every expert, as a sequential walk would give.
+constexpr int kScatterWarps = 8;
+__global__ void __launch_bounds__(kScatterWarps * 32)
+    k_scatter(const int32_t* __restrict__ idx, const float* __restrict__ w, int T, int k, int E,
+              const int* __restrict__ blockcounts, const int* __restrict__ offsets, int* __restrict__ perm,
+              int* __restrict__ slot, float* __restrict__ wperm) {
     extern __shared__ int sm[];
-    int* cursor = sm;            // [E]
-    int* sidx = sm + E;          // [kChunk * k]
+    int* cur = sm;                        // [kScatterWarps][E] per-warp cursors
+    int* sidx = sm + kScatterWarps * E;   // [kChunk * k]
     const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
     const int n = (t1 - t0) * k;
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        cursor[e] = offsets[e] + blockcounts[(size_t)blockIdx.x * E + e];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) cur[i] = 0;
     for (int i = threadIdx.x; i < n; i += blockDim.x) sidx[i] = idx[(size_t)t0 * k + i];
     __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        for (int tl = 0; tl < t1 - t0; ++tl) {
-            for (int j = lane; j < k; j += 32) {
-                const int e = sidx[tl * k + j];
-                const int pos = cursor[e];
-                cursor[e] = pos + 1;
-                sidx[tl * k + j] = pos;  // slot, written back below
-            }
-            __syncwarp();
+    const int w0 = warp * (kChunk / kScatterWarps);
+    const int w1 = min(t1 - t0, w0 + kChunk / kScatterWarps);
+    for (int i = w0 * k + lane; i < w1 * k; i += 32) atomicAdd(&cur[warp * E + sidx[i]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {  // exclusive prefix over the warps
+        int run = offsets[e] + blockcounts[(size_t)blockIdx.x * E + e];
+        for (int q = 0; q < kScatterWarps; ++q) {
+            const int c = cur[q * E + e];
+            cur[q * E + e] = run;
+            run += c;
         }
+    }
+    __syncthreads();
+    int* mycur = cur + warp * E;
+    for (int tl = w0; tl < w1; ++tl) {
+        for (int j = lane; j < k; j += 32) {
+            const int e = sidx[tl * k + j];
+            const int pos = mycur[e];
+            mycur[e] = pos + 1;
+            sidx[tl * k + j] = pos;  // slot, written out below
+        }
+        __syncwarp();
     }
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -229,7 +250,7 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
                               reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
                               reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
                               reinterpret_cast<WsStats*>(ws + p.stats));
-    const size_t scatter_smem = (size_t)(E + kChunk * k) * sizeof(int);
+    const size_t scatter_smem = (size_t)(kScatterWarps * E + kChunk * k) * sizeof(int);
     if (scatter_smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
         if (e != cudaSuccess) return e;

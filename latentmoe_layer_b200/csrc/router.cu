@@ -58,7 +58,45 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
     const int per = E / G;
     if (G > 1) {
         F gs = ninf;
-        if (lane < G) {
+        if (per % 32 == 0) {
+            // group g = i / m for every lane (m = per / 32): lane-local top-2, then warp top-2
+            const int m = per >> 5;
+            for (int g = 0; g < G; ++g) {
+                F a = ninf, b = ninf;
+                for (int i = g * m; i < (g + 1) * m; ++i) {
+                    const F v = c[lane + (i << 5)];
+                    if (v > a) {
+                        b = a;
+                        a = v;
+                    } else if (v > b) {
+                        b = v;
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const F oa = __shfl_xor_sync(0xFFFFFFFFu, a, off), ob = __shfl_xor_sync(0xFFFFFFFFu, b, off);
+                    const F na = fmax(a, oa);
+                    b = a >= oa ? fmax(b, oa) : fmax(a, ob);
+                    a = na;
+                }
+                if (lane == g) gs = a + b;
+            }
+        } else if (32 % per == 0) {
+            // each row of 32 lanes holds 32 / per whole groups, `per` consecutive lanes each
+            const int gpr = 32 / per;
+            for (int i = 0; i < ((E + 31) >> 5); ++i) {
+                const int e = lane + (i << 5);
+                F a = e < E ? c[e] : ninf, b = ninf;
+                for (int off = per >> 1; off > 0; off >>= 1) {
+                    const F oa = __shfl_xor_sync(0xFFFFFFFFu, a, off), ob = __shfl_xor_sync(0xFFFFFFFFu, b, off);
+                    const F na = fmax(a, oa);
+                    b = a >= oa ? fmax(b, oa) : fmax(a, ob);
+                    a = na;
+                }
+                const F sum = __shfl_sync(0xFFFFFFFFu, a + b, (lane % gpr) * per);
+                if (lane < G && lane / gpr == i) gs = sum;
+            }
+        } else if (lane < G) {
             F a = ninf, b = ninf;
             for (int e = lane * per; e < (lane + 1) * per; ++e) {
                 F v = c[e];
@@ -219,23 +257,38 @@ __global__ void __launch_bounds__(256)
             __syncthreads();
             cur = t;
         }
-        for (int e = ch * kEChunk + warp; e < min(E, (ch + 1) * kEChunk); e += 8) {
-            const uint16_t* wrow = wr + (size_t)e * H;
-            double acc = 0.0;
-            for (int h = lane * 8; h < H; h += 256) {
-                const uint4 pk = *reinterpret_cast<const uint4*>(wrow + h);
-                const double2* xv = reinterpret_cast<const double2*>(xrow + h);
-                const uint32_t u[4] = {pk.x, pk.y, pk.z, pk.w};
+        // each warp: 8 experts of the chunk, 4 rows streamed at once (independent loads)
+        const int e_end = min(E, (ch + 1) * kEChunk);
+        for (int e0 = ch * kEChunk + warp * 8; e0 < min(e_end, ch * kEChunk + warp * 8 + 8); e0 += 4) {
+            const uint16_t* wrow[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const double2 xx = xv[q];
-                    acc = fma(xx.x, (double)__uint_as_float(u[q] << 16), acc);
-                    acc = fma(xx.y, (double)__uint_as_float(u[q] & 0xFFFF0000u), acc);
+            for (int j = 0; j < 4; ++j) wrow[j] = wr + (size_t)min(e0 + j, E - 1) * H;
+            double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+            for (int h = lane * 8; h < H; h += 256) {
+                uint4 pk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) pk[j] = __ldg(reinterpret_cast<const uint4*>(wrow[j] + h));
+                const double2* xv = reinterpret_cast<const double2*>(xrow + h);
+                double2 xx[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xx[q] = xv[q];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t u[4] = {pk[j].x, pk[j].y, pk[j].z, pk[j].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[j][q & 1] = fma(xx[q].x, (double)__uint_as_float(u[q] << 16), acc[j][q & 1]);
+                        acc[j][q & 1] = fma(xx[q].y, (double)__uint_as_float(u[q] & 0xFFFF0000u), acc[j][q & 1]);
+                    }
                 }
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-            if (lane == 0) out[(size_t)t * E + e] = acc;
+            for (int j = 0; j < 4; ++j) {
+                double a = acc[j][0] + acc[j][1];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+                if (lane == 0 && e0 + j < e_end) out[(size_t)t * E + e0 + j] = a;
+            }
         }
     }
 }

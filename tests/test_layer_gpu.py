@@ -174,23 +174,24 @@ def test_route_entry_point_matches_forward():
     assert int(counts.sum()) == RAGGED.T * RAGGED.k
 
 
-def test_zero_margin_shows_fp32_edge_cases_are_rechecked():
-    """With the near-edge margin forced to 0 no token is re-checked in fp64; the
-    default margin re-checks a few and routing is then exact on every token."""
+def test_near_edge_recheck_margin():
+    """Routing is exact with the default margin; with a wide margin many tokens go
+    through the fp64 re-decision and routing is still exact; with no margin no
+    token is re-checked (the count of tokens that then differ is reported)."""
     import torch
     shape = replace(ULTRA_DECODE, name="ultra_1k", T=1024)
     layer, dev = H.device_layer(shape)
-    idx, _, _ = layer.route(dev["x"])
-    torch.cuda.synchronize()
-    st = layer.stats()
     host = H.host_weights_for(shape, dev, [])
     ri, _ = H.oracle_route(shape, H.host_x(shape, dev, np.arange(shape.T)), host)
-    assert np.array_equal(idx.cpu().numpy(), ri)
-    layer.set_option(2, 0)
-    idx0, _, _ = layer.route(dev["x"])
-    torch.cuda.synchronize()
-    st0 = layer.stats()
-    mism = int((idx0.cpu().numpy() != ri).any(1).sum())
-    print("flagged(default)=%d flagged(0)=%d mismatching tokens without re-check=%d" %
-          (st.flagged_tokens, st0.flagged_tokens, mism))
-    assert st0.flagged_tokens == 0 and st.flagged_tokens > 0
+    flagged = {}
+    for name, delta_1e9 in (("default", None), ("wide", 40000), ("none", 0)):
+        if delta_1e9 is not None:
+            layer.set_option(2, delta_1e9)
+        idx, _, _ = layer.route(dev["x"])
+        torch.cuda.synchronize()
+        flagged[name] = layer.stats().flagged_tokens
+        mism = int((idx.cpu().numpy() != ri).any(1).sum())
+        print("margin %-7s flagged=%d tokens differing from the oracle=%d" % (name, flagged[name], mism))
+        if name != "none":
+            assert mism == 0
+    assert flagged["wide"] > 0 and flagged["none"] == 0
