@@ -110,6 +110,22 @@ def expert_gemm_work(w, distinct):
     return flops, weight_bytes + act_bytes
 
 
+def replica_x_offset(rank: int, shape) -> int:
+    """First element of rank's x in the generator's x stream: replica r processes
+    tokens r*T .. (r+1)*T - 1, so the ranks together process N*T distinct tokens."""
+    return rank * shape.T * shape.H
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time (identity on one process)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -128,10 +144,11 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch):
         import ctypes
         stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         n = shape.T * shape.H
+        off = replica_x_offset(rank, shape)
         if shape.x_f32:
-            lib.synth_cuda_fill_normal_f32(dev["x"].data_ptr(), n, 0, synth.TID_X, 1.0, rank * n, stream)
+            lib.synth_cuda_fill_normal_f32(dev["x"].data_ptr(), n, 0, synth.TID_X, 1.0, off, stream)
         else:
-            lib.synth_cuda_fill_normal_bf16(dev["x"].data_ptr(), n, 0, synth.TID_X, 1.0, rank * n, stream)
+            lib.synth_cuda_fill_normal_bf16(dev["x"].data_ptr(), n, 0, synth.TID_X, 1.0, off, stream)
         if shape.skew_hot:
             dev["x"][:, 0] = 1.0
     layer = lm.LatentMoE(shape, dev, shape.T, x_f32=shape.x_f32)
@@ -171,45 +188,70 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch):
         dist.barrier()
     clk = clocks.stop()
     lm.latentmoe_set_profile_events(layer.h, None, 0)
-    ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dist, "cuda")
     stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, name in enumerate(STAGES)}
     st = layer.stats()
 
-    # end to end through the public call with host buffers: H2D x, forward, D2H y
+    # End to end through the public call with host buffers: every step copies its
+    # x from pinned host memory to the device, runs the layer and copies y back.
+    # Copies run on their own streams, double-buffered, so step i's compute
+    # overlaps step i+1's upload and step i-1's download (as a serving loop would).
     xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     xh.copy_(x)
     yh = torch.empty((shape.T, shape.H), dtype=torch.float32, pin_memory=True)
-    xd = torch.empty_like(x)
-    for _ in range(max(1, warmup)):
-        xd.copy_(xh, non_blocking=True)
-        layer.forward(xd, y)
-        yh.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    e_steps = max(1, min(steps, 50))
+    xd = [torch.empty_like(x) for _ in range(2)]
+    yd = [torch.empty_like(y) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n):
+        h2d_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        d2h_done = [torch.cuda.Event() for _ in range(2)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        up.wait_event(start)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[b])
+                xd[b].copy_(xh, non_blocking=True)
+                h2d_done[b].record(up)
+            comp.wait_event(h2d_done[b])
+            if i >= 2:
+                comp.wait_event(d2h_done[b])
+            layer.forward(xd[b], yd[b])
+            comp_done[b].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[b])
+                yh.copy_(yd[b], non_blocking=True)
+                d2h_done[b].record(down)
+        comp.wait_stream(down)
+        end.record(comp)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    e2e_run(max(2, warmup))
+    e_steps = max(2, min(steps, 50))
     if dist is not None:
         dist.barrier()
-    t_start.record()
-    for _ in range(e_steps):
-        xd.copy_(xh, non_blocking=True)
-        layer.forward(xd, y)
-        yh.copy_(y, non_blocking=True)
-    t_end.record()
-    torch.cuda.synchronize()
-    e_ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e2e_run(e_steps), dist, "cuda")
     res = {
         "ms": ms, "stage_ms": stage_ms, "stats": st, "clocks": clk, "e2e_ms": e_ms, "e2e_steps": e_steps,
         "h2d": x.numel() * x.element_size(), "d2h": y.numel() * 4, "layer": layer, "dev": dev,
     }
     return res
+
+
+# DRAM bytes per assignment of the expert up GEMM, from an ncu capture of this
+# kernel on the probe_e64 workload (2.027 GB for 45 056 assignments; the same
+# tile shapes and rows per expert as ultra_prefill). Traffic grows with the
+# assignments (rows) and, at ~704 rows per expert, with the experts in the same
+# ratio. Reset to None when that kernel changes.
+UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT = 2.027e9 / 45056
 
 
 def roofline_for(shape, res, peaks, peak_src, prefill: bool):
@@ -222,7 +264,10 @@ def roofline_for(shape, res, peaks, peak_src, prefill: bool):
         peak = peaks["bf16_tflops_sustained"]
         return {"kernel": name, "bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(ach / peak, 4), "peak_kind": "%s sustained bf16" % peak_src,
-                "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                "traffic": (round(UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT * shape.T * shape.k)
+                            if name == "expert_up_gemm" and UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT else None),
+                "traffic_note": "ncu capture of the same kernel on probe_e64, scaled by assignments",
                 "algorithmic_per_launch": flops, "launch_ms": round(kms, 4)}
     ach = byts / (kms * 1e-3) / 1e9
     peak = peaks["hbm_gbs"]
