@@ -118,8 +118,9 @@ const char* latentmoe_status_string(lmoe_status s);
 
 /* ---- diagnostics --------------------------------------------------------- */
 typedef enum {
-    LMOE_OPT_GEMM_PATH = 0,      /* 0 auto, 1 tcgen05 prefill tiles, 2 tcgen05 decode (swap-AB)
-                                    tiles, 3 SIMT fp32-accumulate kernels (validation)           */
+    LMOE_OPT_GEMM_PATH = 0,      /* 0 auto, 1 tcgen05 prefill tiles (128 x BN per SM), 2 tcgen05
+                                    decode (swap-AB) tiles, 3 SIMT fp32 kernels (validation),
+                                    4 prefill tiles of 256 x 256 on 2-SM pairs (cta_group::2)     */
     LMOE_OPT_ROUTER_FP64_ALL = 1,/* 1: every token's logits recomputed in fp64 (validation)      */
     LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin for the fp64 re-check, in 1e-9 units        */
     LMOE_OPT_SPIN_LIMIT = 3      /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */

@@ -22,7 +22,7 @@ LMOE_OK, LMOE_ERR_INVALID_ARG, LMOE_ERR_UNSUPPORTED, LMOE_ERR_WORKSPACE, LMOE_ER
 LMOE_BF16, LMOE_FP32 = 0, 1
 LMOE_MODE_BF16, LMOE_MODE_FP32 = 0, 1
 OPT_GEMM_PATH, OPT_ROUTER_FP64_ALL, OPT_FLAG_DELTA, OPT_SPIN_LIMIT = range(4)
-GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
+GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",

@@ -93,6 +93,7 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     p.pfx128 = take((E + 1) * 4);
     p.pfx64 = take((E + 1) * 4);
     p.pfxdec = take((E + 1) * 4);
+    p.pfx256 = take((E + 1) * 4);
     p.blockcounts = take((size_t)p.nblk * E * 4);
     p.perm = take(A * 4);
     p.slot = take(A * 4);
@@ -178,6 +179,8 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
     for (int i = 0; i < nprob; ++i) swap = swap && probs[i].n % 128 == 0;
     const int bn = swap ? kDecodeTN : pick_bn(ns, nprob);
     if (bn == 0) return cudaErrorInvalidValue;
+    // 256 x 256 tiles on 2-SM pairs (option 4): each CTA of the pair loads 128 rows of B
+    const bool pair = !swap && bn == 256 && c.h->gemm_path == 4;
     CUtensorMap maps[8];
     int nm = 0;
     for (int i = 0; i < nprob; ++i)
@@ -186,7 +189,7 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
             if (!encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? kDecodeTN : kBM))
                 return cudaErrorInvalidValue;
             probs[i].a_map[sg] = nm++;
-            if (!encode_bf16(&maps[nm], b[i][sg].ptr, b[i][sg].rows, K, swap ? kBM : bn))
+            if (!encode_bf16(&maps[nm], b[i][sg].ptr, b[i][sg].rows, K, swap ? kBM : pair ? 128 : bn))
                 return cudaErrorInvalidValue;
             probs[i].b_map[sg] = nm++;
         }
@@ -201,6 +204,7 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
         probs[i].out_map = nm++;
     }
     if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
+    if (pair) return launch_gemm_tc_pair(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
     return launch_gemm_tc(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
 }
 
@@ -299,11 +303,12 @@ Ctx make_ctx(lmoe_handle* h, const Plan& p, void* ws, void* stream) {
     c.r.pfx128 = reinterpret_cast<const int*>(c.ws + p.pfx128);
     c.r.pfx64 = reinterpret_cast<const int*>(c.ws + p.pfx64);
     c.r.pfxdec = reinterpret_cast<const int*>(c.ws + p.pfxdec);
+    c.r.pfx256 = reinterpret_cast<const int*>(c.ws + p.pfx256);
     c.r.E = h->cfg.num_experts;
     c.err = &reinterpret_cast<WsStats*>(c.ws + p.stats)->device_error;
     const lmoe_config& cf = h->cfg;
     c.simt = h->gemm_path == 3 || cf.mode == LMOE_MODE_FP32;
-    if (h->gemm_path == 1) c.decode = false;
+    if (h->gemm_path == 1 || h->gemm_path == 4) c.decode = false;
     else if (h->gemm_path == 2) c.decode = true;
     else c.decode = (long long)p.T * cf.top_k <= 64LL * cf.num_experts;  // <= 64 rows per expert on average
     return c;
@@ -499,7 +504,7 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
     if (!h) return LMOE_ERR_INVALID_ARG;
     switch (opt) {
         case LMOE_OPT_GEMM_PATH:
-            if (v < 0 || v > 3) return LMOE_ERR_INVALID_ARG;
+            if (v < 0 || v > 4) return LMOE_ERR_INVALID_ARG;
             h->gemm_path = (int)v;
             return LMOE_OK;
         case LMOE_OPT_ROUTER_FP64_ALL:

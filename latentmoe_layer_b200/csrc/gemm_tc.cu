@@ -73,6 +73,7 @@ struct TileInfo {
     int rows;    // valid activation rows in this tile
     int wrow0;   // first weight row (row of B)
     int col0;    // first output column
+    bool half;   // non-swapped tile with <= 64 valid rows: M = 64 MMAs (the expert's ragged tail)
 };
 
 template <int BN, bool kSwap>
@@ -136,6 +137,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         ti.rows = min(S::kActRows, end - ti.row0);
         ti.col0 = ct * S::kOutCols;
         ti.wrow0 = e * pr.b_rows_per_expert + ti.col0;
+        ti.half = !kSwap && ti.rows <= 64;
         return ti;
     }
     int p = 0;
@@ -161,6 +163,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
     ti.rows = min(S::kActRows, pr.m_rows - ti.row0);
     ti.col0 = ct * S::kOutCols;
     ti.wrow0 = ti.col0;
+    ti.half = !kSwap && ti.rows <= 64;
     return ti;
 }
 
@@ -353,13 +356,16 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
             if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+        constexpr uint32_t idesc_full = idesc_bf16_f32(128, BN);
+        constexpr uint32_t idesc_half = idesc_bf16_f32(64, BN);
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
             const int kb_total = tile_kblocks(P.prob[ti.p]);
+            // M = 64 puts D rows 16q..16q+15 in TMEM lanes 32q..32q+15 (q = lane quarter)
+            const uint32_t idesc = ti.half ? idesc_half : idesc_full;
             for (int kb0 = 0; kb0 < kb_total && ok; kb0 += CK) {
                 // next chunk accumulator must have been drained by the epilogue
                 if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, P.spin, err)) {
@@ -465,8 +471,10 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
 #pragma unroll
             for (int i = 0; i < CW; ++i) acc[i] = (float)accd[i];
 #endif
-            const CUtensorMap* omap = pr.out_map >= 0 ? &P.maps[pr.out_map] : nullptr;
-            epilogue_store<BN, kSwap, CW>(pr, ti, lane_row, c0, acc, omap, sOut + ew * S::kStageOutBytes);
+            const CUtensorMap* omap = pr.out_map >= 0 && !ti.half ? &P.maps[pr.out_map] : nullptr;
+            // half tiles: only lanes 0..15 of each quarter carry rows (row = 16q + lane)
+            const int row_in_tile = ti.half ? (lane < 16 ? q * 16 + lane : 1 << 20) : lane_row;
+            epilogue_store<BN, kSwap, CW>(pr, ti, row_in_tile, c0, acc, omap, sOut + ew * S::kStageOutBytes);
         }
         if (!kSwap && lane == 0) bulk_wait_all();  // this warp's bulk stores are complete
     }
@@ -475,6 +483,266 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
         tc_fence_after();
         tmem_dealloc(tmem_base, S::kTmemCols);
     }
+}
+
+// ---------------------------------------------------------------- 2-SM pairs
+// (Selected with LMOE_OPT_GEMM_PATH = 4; measured no faster than the single-SM
+// tiles on this layer, whose steady state is set by the 1 kW power cap.)
+// A cluster of two CTAs on neighbouring SMs computes one 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256). Each CTA stages its own 128 A
+// rows and its own half (128 rows) of B, 32 KB per k-block instead of the
+// 48 KB a single CTA needs for 128 x 256, which keeps each SM's shared-memory
+// traffic (TMA writes plus MMA operand reads) within its bandwidth and leaves
+// room for 6 pipeline stages. The leader CTA (rank 0) issues the MMAs and
+// commits them to barriers in both CTAs; each CTA drains its own 128 TMEM
+// lanes, adds the K chunks in fp32 registers exactly as the single-CTA kernel
+// does, and writes its own rows. Loads use the cta_group::2 form that counts
+// completion on the leader's barrier; nothing is multicast.
+struct PairShape {
+    static constexpr int BN = 256;
+    static constexpr int kXBytes = 128 * kBK * 2;   // this CTA's 128 A rows
+    static constexpr int kYBytes = 128 * kBK * 2;   // this CTA's 128 rows of B
+    static constexpr int kStageBytes = kXBytes + kYBytes;
+    static constexpr int kChunkKB = LMOE_CHUNK_KB;
+    static constexpr int kBufs = 2;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr int kEpiWarps = 8;
+    static constexpr int kColsPerThread = 128;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kStageOutBytes = 4096;
+    static constexpr int kGroupM = 8;
+};
+
+__device__ __forceinline__ int pair_total_tiles(const TcParams& P) {
+    if (P.prob[0].grouped) return P.r.pfx256[P.r.E] * (P.prob[0].n / PairShape::BN);
+    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
+}
+
+// Pair tile t -> this CTA's half: rows row0 .. row0+rows-1 (rows may be <= 0
+// for the second CTA of a short tile), B rows wrow0 .. wrow0+127, output
+// columns col0 .. col0+255.
+__device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32_t rank) {
+    int p = 0, prow0, prows, ct, wbase = 0;
+    if (P.prob[0].grouped) {
+        const GemmProblem& pr = P.prob[0];
+        const int nct = pr.n / PairShape::BN;
+        const int mt = t / nct;
+        ct = t % nct;
+        const int* pfx = P.r.pfx256;
+        int lo = 0, hi = P.r.E;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(&pfx[mid]) <= mt) lo = mid;
+            else hi = mid;
+        }
+        const int off = __ldg(&P.r.offsets[lo]), end = __ldg(&P.r.offsets[lo + 1]);
+        prow0 = off + (mt - __ldg(&pfx[lo])) * 256;
+        prows = min(256, end - prow0);
+        wbase = lo * pr.b_rows_per_expert;
+    } else {
+        if (P.nprob > 1 && t >= P.dense_tiles[0]) {
+            t -= P.dense_tiles[0];
+            p = 1;
+        }
+        const GemmProblem& pr = P.prob[p];
+        const int nct = pr.n / PairShape::BN;
+        const int mtc = (pr.m_rows + 255) / 256;
+        const int g = t / (PairShape::kGroupM * nct), r = t % (PairShape::kGroupM * nct);
+        const int ms = min(PairShape::kGroupM, mtc - g * PairShape::kGroupM);
+        const int mt = g * PairShape::kGroupM + r % ms;
+        ct = r / ms;
+        prow0 = mt * 256;
+        prows = min(256, pr.m_rows - prow0);
+    }
+    TileInfo ti;
+    ti.p = p;
+    ti.row0 = prow0 + (int)rank * 128;
+    ti.rows = min(128, prows - (int)rank * 128);
+    ti.col0 = ct * PairShape::BN;
+    ti.wrow0 = wbase + ti.col0 + (int)rank * 128;
+    ti.half = false;
+    return ti;
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(PairShape::kThreads, 1) k_gemm_tc_pair(const __grid_constant__ TcParams P) {
+    using S = PairShape;
+    constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread, BN = S::BN;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base_u32 = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
+    uint8_t* sX = smem;
+    uint8_t* sY = smem + STAGES * S::kXBytes;
+    uint8_t* sOut = sY + STAGES * S::kYBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + S::kEpiWarps * S::kStageOutBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* cfull = empty + STAGES;
+    uint64_t* cempty = cfull + NB;
+    uint64_t* done = cempty + NB;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&cfull[b], 1);
+            mbar_init(&cempty[b], 2 * S::kEpiWarps);  // both CTAs' epilogue warps
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, S::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers and TMEM of both CTAs are ready
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntiles = pair_total_tiles(P);
+    int* err = P.err;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0, issued = 0, issued_par = 0;
+        bool ok = true;
+        for (int t = pair; t < ntiles && ok; t += npairs) {
+            const TileInfo ti = pair_decode(P, t, rank);
+            const GemmProblem& pr = P.prob[ti.p];
+            for (int sg = 0; sg < pr.nseg && ok; ++sg) {
+                const CUtensorMap* amap = &P.maps[pr.a_map[sg]];
+                const CUtensorMap* bmap = &P.maps[pr.b_map[sg]];
+                const int kb_n = pr.kdim[sg] / kBK;
+                for (int kb = 0; kb < kb_n; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, P.spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+                    const uint32_t lbar = mapa_shared(&full[stage], 0);
+                    tma_load_2d_pair(sX + stage * S::kXBytes, amap, lbar, kb * kBK, ti.row0);
+                    tma_load_2d_pair(sY + stage * S::kYBytes, bmap, lbar, kb * kBK, ti.wrow0);
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        // the leader's full barriers count both CTAs' bytes: waiting on them drains
+        // every load of the pair before either CTA can pass the final cluster barrier
+        if (leader)
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, bphase = 0;
+        bool ok = true;
+        for (int t = pair; t < ntiles && ok; t += npairs) {
+            const TileInfo ti = pair_decode(P, t, rank);
+            const int kb_total = tile_kblocks(P.prob[ti.p]);
+            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += CK) {
+                if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, P.spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+                const int kb1 = min(kb_total, kb0 + CK);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_sw128(smem_u32(sX + stage * S::kXBytes));
+                    const uint64_t bdesc = sdesc_sw128(smem_u32(sY + stage * S::kYBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16_pair(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                                       (kb > kb0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair_both(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair_both(&cfull[buf]);
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+        }
+        umma_commit_pair_self(done);
+        mbar_wait_bounded(done, 0, 1u << 26, err);
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int q = warp & 3;
+        const int c0 = (ew >> 2) * CW;
+        const int lane_row = q * 32 + lane;
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (int t = pair; t < ntiles && ok; t += npairs) {
+            const TileInfo ti = pair_decode(P, t, rank);
+            const GemmProblem& pr = P.prob[ti.p];
+            const int kb_total = tile_kblocks(pr);
+            float acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = 0.f;
+            for (int kb0 = 0; kb0 < kb_total; kb0 += CK) {
+                if (!mbar_wait_bounded(&cfull[buf], bphase, P.spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0);
+#pragma unroll
+                for (int c = 0; c < CW; c += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(taddr + (uint32_t)c, r0);
+                    tmem_ld16(taddr + (uint32_t)(c + 16), r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[c + i] += __uint_as_float(r0[i]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[c + 16 + i] += __uint_as_float(r1[i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(&cempty[buf], 0));
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            const CUtensorMap* omap = pr.out_map >= 0 ? &P.maps[pr.out_map] : nullptr;
+            epilogue_store<BN, false, CW>(pr, ti, lane_row, c0, acc, omap, sOut + ew * S::kStageOutBytes);
+        }
+        if (lane == 0) bulk_wait_all();
+    }
+    __syncthreads();
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs done with TMEM; the leader's MMAs have completed
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, S::kTmemCols);
 }
 
 template <int BN, int STAGES, bool kSwap>
@@ -551,6 +819,44 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
         case 64: return launch_impl<64, 8, false>(P, grid, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+                                const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    constexpr int STAGES = 6;
+    using S = PairShape;
+    constexpr size_t smem = 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 256;
+    static_assert(smem <= 232448, "shared memory");
+    static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 256, "barrier area");
+    TcParams P;
+    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
+    int pairs = tc_num_sms() / 2;
+    if (!probs[0].grouped) {
+        long long tiles = 0;
+        for (int i = 0; i < nprob; ++i) {
+            P.dense_tiles[i] = ((probs[i].m_rows + 255) / 256) * (probs[i].n / S::BN);
+            tiles += P.dense_tiles[i];
+        }
+        if (tiles < pairs) pairs = (int)tiles;
+        if (pairs < 1) return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc_pair<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_gemm_tc_pair<STAGES>, P);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,

@@ -61,13 +61,14 @@ struct DeviceRouting {
     const int* pfx128;      // [E+1] prefix of ceil(count/128)
     const int* pfx64;       // [E+1] prefix of ceil(count/64)
     const int* pfxdec;      // [E+1] prefix of ceil(count/kDecodeTN)
+    const int* pfx256;      // [E+1] prefix of ceil(count/256) (2-SM pair tiles)
     int E;
 };
 
 // Workspace carving for one call.
 struct Plan {
     size_t total;
-    size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, blockcounts, perm,
+    size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, blockcounts, perm,
         slot, wperm, xbf, z, zperm, aperm, o, comb, as;
     int T, A, nblk;
 };
@@ -93,6 +94,8 @@ cudaError_t launch_gemm_simt(const GemmProblem* probs, int nprob, bool a_f32, co
                              cudaStream_t s);
 cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
                            const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
+cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+                                const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
 cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
                                   const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* err, unsigned spin_limit, cudaStream_t s);

@@ -79,7 +79,7 @@ __device__ void block_scan4(int4& v, int4* warp_tot) {
 __global__ void __launch_bounds__(1024)
     k_scan(int* __restrict__ blockcounts, int nblk, int E, int* __restrict__ counts, int32_t* __restrict__ counts_out,
            int* __restrict__ offsets, int* __restrict__ pfx128, int* __restrict__ pfx64, int* __restrict__ pfxdec,
-           WsStats* __restrict__ st) {
+           int* __restrict__ pfx256, WsStats* __restrict__ st) {
     __shared__ int4 warp_tot[32];
     __shared__ int red[2];
     const int e = threadIdx.x;
@@ -107,6 +107,14 @@ __global__ void __launch_bounds__(1024)
     int4 v = make_int4(run, (run + 127) / 128, (run + 63) / 64, (run + kDecodeTN - 1) / kDecodeTN);
     int4 incl = v;
     block_scan4(incl, warp_tot);
+    __syncthreads();
+    int4 v2 = make_int4((run + 255) / 256, 0, 0, 0);
+    int4 incl2 = v2;
+    block_scan4(incl2, warp_tot);
+    if (e < E) {
+        pfx256[e] = incl2.x - v2.x;
+        if (e == E - 1) pfx256[E] = incl2.x;
+    }
     if (e < E) {
         offsets[e] = incl.x - v.x;
         pfx128[e] = incl.y - v.y;
@@ -249,7 +257,7 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
     k_scan<<<1, 1024, 0, s>>>(bc, p.nblk, E, reinterpret_cast<int*>(ws + p.counts), counts_out,
                               reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
                               reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
-                              reinterpret_cast<WsStats*>(ws + p.stats));
+                              reinterpret_cast<int*>(ws + p.pfx256), reinterpret_cast<WsStats*>(ws + p.stats));
     const size_t scatter_smem = (size_t)(kScatterWarps * E + kChunk * k) * sizeof(int);
     if (scatter_smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);

@@ -15,7 +15,7 @@ import helpers as H
 
 pytestmark = pytest.mark.gpu
 
-GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT = range(4)
+GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 # several tiles and ragged tails in every dimension the kernels tile
 RAGGED = LayerShape("ragged", T=333, H=512, L=256, E=64, k=6, G=4, Gk=2, I=384, Is=640)
@@ -53,7 +53,7 @@ def test_tiny_fp32_validation_mode():
     run_and_compare(TINY, mode=1)
 
 
-@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT])
+@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_PREFILL_PAIR, GEMM_DECODE, GEMM_SIMT])
 def test_ragged_bf16(path):
     run_and_compare(RAGGED, mode=0, path=path)
 
@@ -66,7 +66,7 @@ def test_ragged_fp32_validation_mode():
     run_and_compare(RAGGED, mode=1)
 
 
-@pytest.mark.parametrize("path", [GEMM_AUTO, GEMM_PREFILL])
+@pytest.mark.parametrize("path", [GEMM_AUTO, GEMM_PREFILL, GEMM_PREFILL_PAIR])
 def test_nano_decode_full(path):
     (ma, rf), layer = run_and_compare(NANO_DECODE, mode=0, path=path)
     st = layer.stats()
