@@ -116,6 +116,20 @@ void latentmoe_destroy(lmoe_handle* h);
 
 const char* latentmoe_status_string(lmoe_status s);
 
+/* Load-balancing step for the bias the router adds to its choice scores
+ * ("Nemotron 3 Ultra 架构 QA", Q5.3: the training framework counts the tokens
+ * each expert received and lowers the bias of overloaded experts; Q5.4 reports
+ * MaxVio). With mean = sum(expert_counts) / E, in fp64:
+ *   bias_out[e] = fp32(bias_in[e] - eta * (expert_counts[e] - mean))
+ *   *maxvio_out = (max_e expert_counts[e] - mean) / mean   (0 if no token)
+ * expert_counts [E] int32 (e.g. the counts latentmoe_route/forward return),
+ * bias_in/bias_out [E] fp32, maxvio_out one double (may be NULL); all device
+ * memory. bias_out may alias bias_in, including the handle's own e_bias: the
+ * handle reads the bias through its pointer, so the next call uses it.
+ * Asynchronous on `stream`. */
+lmoe_status latentmoe_update_bias(lmoe_handle* h, const int32_t* expert_counts, const float* bias_in, float eta,
+                                  float* bias_out, double* maxvio_out, void* stream);
+
 /* ---- diagnostics --------------------------------------------------------- */
 typedef enum {
     LMOE_OPT_GEMM_PATH = 0,      /* 0 auto, 1 tcgen05 prefill tiles (128 x BN per SM), 2 tcgen05

@@ -26,7 +26,7 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
-           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc"]
+           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -79,9 +79,10 @@ def load():
     lib.latentmoe_selftest_bounded_wait.argtypes = [vp]
     lib.latentmoe_set_profile_events.argtypes = [vp, vp, i32]
     lib.latentmoe_route_noalloc.argtypes = [vp, vp, i32, vp, vp, vp, vp]
+    lib.latentmoe_update_bias.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
-              "latentmoe_set_profile_events", "latentmoe_route_noalloc"):
+              "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -137,6 +138,10 @@ def latentmoe_set_profile_events(h, events, n: int) -> int:
 def latentmoe_route_noalloc(h, x, T, idx, w, counts, stream) -> int:
     """Routing with the library's static scratch (no workspace, no allocation)."""
     return load().latentmoe_route_noalloc(h, x, T, idx, w, counts, stream)
+
+
+def latentmoe_update_bias(h, counts, bias_in, eta, bias_out, maxvio, stream) -> int:
+    return load().latentmoe_update_bias(h, counts, bias_in, eta, bias_out, maxvio, stream)
 
 
 def latentmoe_selftest_bounded_wait(h) -> int:
@@ -210,6 +215,13 @@ class LatentMoE:
         if s != LMOE_OK:
             raise LmoeError(s, "latentmoe_route")
         return idx, w, counts
+
+    def update_bias(self, counts, eta: float, maxvio=None):
+        """In-place load-balancing step on this layer's e_bias tensor."""
+        b = self.weights["e_bias"]
+        s = latentmoe_update_bias(self.h, _p(counts), _p(b), float(eta), _p(b), _p(maxvio), self._stream())
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_update_bias")
 
     def stats(self):
         s, st = latentmoe_read_stats(self.h, _p(self._ws))

@@ -534,6 +534,15 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
     return LMOE_OK;
 }
 
+lmoe_status latentmoe_update_bias(lmoe_handle* h, const int32_t* expert_counts, const float* bias_in, float eta,
+                                  float* bias_out, double* maxvio_out, void* stream) {
+    if (!h || !expert_counts || !bias_in || !bias_out || !aligned(expert_counts, 4) || !aligned(bias_in, 4) ||
+        !aligned(bias_out, 4) || (maxvio_out && !aligned(maxvio_out, 8)) || !(eta == eta) || isinf(eta))
+        return LMOE_ERR_INVALID_ARG;
+    return cuda_status(launch_update_bias(expert_counts, bias_in, h->cfg.num_experts, (double)eta, bias_out, maxvio_out,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n) {
     if (!h || (events && n < 8)) return LMOE_ERR_INVALID_ARG;
     h->prof_events = events;

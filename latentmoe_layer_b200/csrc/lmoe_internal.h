@@ -88,6 +88,8 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int 
                                int row_bytes, cudaStream_t s);
 cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
                            cudaStream_t s);
+cudaError_t launch_update_bias(const int32_t* counts, const float* bias_in, int E, double eta, float* bias_out,
+                               double* maxvio, cudaStream_t s);
 cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n,
                                 cudaStream_t s);
 cudaError_t launch_gemm_simt(const GemmProblem* probs, int nprob, bool a_f32, const DeviceRouting& r, int max_rows,

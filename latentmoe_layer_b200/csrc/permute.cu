@@ -241,6 +241,50 @@ __global__ void k_copy_routing(const int* __restrict__ idx, const float* __restr
     }
 }
 
+// Load-balancing bias update ("Nemotron 3 Ultra 架构 QA", Q5.3) and MaxVio (Q5.4):
+// one block; integer reductions are exact, and the fp64 update is written with
+// explicit round-to-nearest multiply and subtract so no fused multiply-add
+// changes its rounding.
+__global__ void __launch_bounds__(1024)
+    k_update_bias(const int32_t* __restrict__ counts, const float* __restrict__ bias_in, int E, double eta,
+                  float* __restrict__ bias_out, double* __restrict__ maxvio) {
+    __shared__ long long s_tot[32];
+    __shared__ int s_max[32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const int c = e < E ? counts[e] : 0;
+    long long t = c;
+    int m = c;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        t += __shfl_xor_sync(0xFFFFFFFFu, t, off);
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    }
+    if (lane == 0) {
+        s_tot[warp] = t;
+        s_max[warp] = m;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        t = s_tot[lane];
+        m = s_max[lane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            t += __shfl_xor_sync(0xFFFFFFFFu, t, off);
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        }
+        if (lane == 0) {
+            s_tot[0] = t;
+            s_max[0] = m;
+        }
+    }
+    __syncthreads();
+    const double mean = (double)s_tot[0] / (double)E;
+    const float b = e < E ? bias_in[e] : 0.f;  // read before any write: bias_out may alias bias_in
+    __syncthreads();
+    if (e < E) bias_out[e] = (float)__dsub_rn((double)b, __dmul_rn(eta, __dsub_rn((double)c, mean)));
+    if (e == 0 && maxvio) *maxvio = mean > 0.0 ? __ddiv_rn(__dsub_rn((double)s_max[0], mean), mean) : 0.0;
+}
+
 inline int grid_cap(long long work, int per_block, int cap) {
     long long g = (work + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -293,6 +337,12 @@ cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStre
     long long n4 = n / 4;
     k_convert<<<grid_cap(n4, 256, 148 * 16), 256, 0, s>>>(reinterpret_cast<const float4*>(x),
                                                           reinterpret_cast<uint2*>(xb), n4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_update_bias(const int32_t* counts, const float* bias_in, int E, double eta, float* bias_out,
+                               double* maxvio, cudaStream_t s) {
+    k_update_bias<<<1, 1024, 0, s>>>(counts, bias_in, E, eta, bias_out, maxvio);
     return cudaGetLastError();
 }
 

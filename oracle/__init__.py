@@ -56,6 +56,8 @@ def _get():
         lib.lmo_logits.argtypes = [vp, vp, vp, i64, vp]
         lib.lmo_route.argtypes = [vp, vp, vp, vp, i64, vp, vp]
         lib.lmo_forward.argtypes = [vp, vp, vp, i64, vp, vp, vp]
+        lib.lmo_update_bias.argtypes = [ctypes.c_int, vp, vp, ctypes.c_double, vp, vp]
+        lib.lmo_update_bias.restype = ctypes.c_int
         for f in (lib.lmo_select, lib.lmo_logits, lib.lmo_route, lib.lmo_forward):
             f.restype = ctypes.c_int
         _lib = lib
@@ -147,3 +149,14 @@ def forward(cfg: LmoCfg, x, wts: dict):
     if rc != 0:
         raise ValueError("oracle forward failed (invalid configuration or missing expert weights)")
     return y, idx, w
+
+
+def update_bias(counts, bias, eta):
+    """Returns (new bias fp32 [E], MaxVio)."""
+    counts = _c(np.asarray(counts, dtype=np.int32), np.int32)
+    bias = _c(np.asarray(bias, dtype=np.float32), np.float32)
+    out = np.zeros_like(bias)
+    mv = ctypes.c_double()
+    _get().lmo_update_bias(len(bias), counts.ctypes.data, bias.ctypes.data, float(eta), out.ctypes.data,
+                           ctypes.byref(mv))
+    return out, mv.value

@@ -240,3 +240,16 @@ int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64
     }
     return bad ? -1 : 0;
 }
+
+/* Bias update and MaxVio ("Nemotron 3 Ultra 架构 QA", Q5.3 and Q5.4). */
+int lmo_update_bias(int E, const int32_t* counts, const float* bias, double eta, float* bias_out, double* maxvio) {
+    long long total = 0, mx = 0;
+    for (int e = 0; e < E; ++e) {
+        total += counts[e];
+        if (counts[e] > mx) mx = counts[e];
+    }
+    const double mean = (double)total / (double)E;
+    for (int e = 0; e < E; ++e) bias_out[e] = (float)((double)bias[e] - eta * ((double)counts[e] - mean));
+    if (maxvio) *maxvio = mean > 0.0 ? ((double)mx - mean) / mean : 0.0;
+    return 0;
+}

@@ -76,6 +76,15 @@ int lmo_route(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, const
 int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64_t n, int32_t* idx, double* w,
                 double* y);
 
+/* Load-balancing bias update ("Nemotron 3 Ultra 架构 QA", Q5.3: the training
+ * framework counts the tokens each expert received and moves the bias against
+ * the overload): mean = sum(counts) / E,
+ *   bias_out[e] = fp32(bias[e] - eta * (counts[e] - mean))      (fp64 inside)
+ * and MaxVio (Q5.4, load violation relative to the ideal load)
+ *   = (max_e counts[e] - mean) / mean   (0 when no token was routed).
+ * bias_out may alias bias. Returns 0. */
+int lmo_update_bias(int E, const int32_t* counts, const float* bias, double eta, float* bias_out, double* maxvio);
+
 #ifdef __cplusplus
 }
 #endif

@@ -347,3 +347,30 @@ def test_flop_and_param_counts_match_page_figures():
     }
     for name, (val, tol) in g.items():
         assert abs(got[name] - val) <= tol * val, (name, got[name])
+
+
+# ------------------------------------------------------------------ bias update (Q5.3, Q5.4)
+def test_bias_update_uniform_load_is_a_fixed_point(built_oracle):
+    b = synth.uniform_f32(32, 0, 3, -0.1, 0.1)
+    nb, mv = built_oracle.update_bias(np.full(32, 7), b, 0.01)
+    assert np.array_equal(nb, b) and mv == 0.0
+
+
+def test_bias_update_moves_against_overload(built_oracle):
+    counts = np.array([10, 0, 5, 5], dtype=np.int32)   # mean 5
+    b = np.zeros(4, np.float32)
+    nb, mv = built_oracle.update_bias(counts, b, 0.001)
+    assert nb[0] < 0 < nb[1] and nb[2] == nb[3] == 0.0
+    np.testing.assert_allclose(nb, np.float32([-0.005, 0.005, 0.0, 0.0]), rtol=1e-6)
+    assert mv == 1.0                                       # (10 - 5) / 5
+    # the deviations sum to zero, so the mean bias does not move (up to fp32 rounding)
+    rng = np.random.default_rng(1)
+    counts = rng.integers(0, 100, 64).astype(np.int32)
+    b = rng.uniform(-0.1, 0.1, 64).astype(np.float32)
+    nb, _ = built_oracle.update_bias(counts, b, 1e-4)
+    assert abs(float(nb.astype(np.float64).sum() - b.astype(np.float64).sum())) < 64 * 1e-8
+
+
+def test_bias_update_empty_batch(built_oracle):
+    nb, mv = built_oracle.update_bias(np.zeros(8, np.int32), np.ones(8, np.float32), 0.5)
+    assert np.array_equal(nb, np.ones(8, np.float32)) and mv == 0.0
