@@ -111,6 +111,19 @@ lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_
 lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, void* ws, size_t ws_bytes,
                               void* stream, int32_t* topk_idx, float* topk_w, int32_t* expert_counts);
 
+/* The layer inside its pre-norm residual block ("Nemotron 3 Ultra 架构 QA",
+ * Q2.1: each mixer sits behind a pre-norm and a residual; Q2.8: the RMSNorm
+ * upcasts, multiplies by rsqrt(mean(x^2) + eps), rounds back, scales by gamma):
+ *   xn = bf16(gamma * bf16(x / sqrt(mean_h x^2 + eps)))      (fp64 inside)
+ *   y  = x + layer(xn)                                         (fp32)
+ * x [T, H] bf16 (the handle must have x_dtype LMOE_BF16, else
+ * LMOE_ERR_UNSUPPORTED), norm_w = gamma [H] bf16, norm_eps >= 0 (1e-5 on the
+ * pages). Same workspace and optional routing outputs as latentmoe_forward;
+ * the routing is that of xn. */
+lmoe_status latentmoe_forward_block(lmoe_handle* h, const void* x, int T, const void* norm_w, float norm_eps,
+                                    float* y, void* ws, size_t ws_bytes, void* stream, int32_t* topk_idx,
+                                    float* topk_w, int32_t* expert_counts);
+
 /* Releases the handle (host memory only). */
 void latentmoe_destroy(lmoe_handle* h);
 

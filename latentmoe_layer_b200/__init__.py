@@ -26,7 +26,7 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
-           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias"]
+           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias", "latentmoe_forward_block"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -80,9 +80,11 @@ def load():
     lib.latentmoe_set_profile_events.argtypes = [vp, vp, i32]
     lib.latentmoe_route_noalloc.argtypes = [vp, vp, i32, vp, vp, vp, vp]
     lib.latentmoe_update_bias.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp]
+    lib.latentmoe_forward_block.argtypes = [vp, vp, i32, vp, ctypes.c_float, vp, vp, sz, vp, vp, vp, vp]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
-              "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias"):
+              "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias",
+              "latentmoe_forward_block"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -115,6 +117,10 @@ def latentmoe_route(h, x, T, idx, w, counts, ws, ws_bytes, stream):
 
 def latentmoe_forward(h, x, T, y, ws, ws_bytes, stream, idx=None, w=None, counts=None):
     return load().latentmoe_forward(h, x, T, y, ws, ws_bytes, stream, idx, w, counts)
+
+
+def latentmoe_forward_block(h, x, T, norm_w, norm_eps, y, ws, ws_bytes, stream, idx=None, w=None, counts=None):
+    return load().latentmoe_forward_block(h, x, T, norm_w, norm_eps, y, ws, ws_bytes, stream, idx, w, counts)
 
 
 def latentmoe_destroy(h):
@@ -201,6 +207,19 @@ class LatentMoE:
         s = latentmoe_forward(self.h, _p(x), T, _p(y), _p(ws), ws.numel(), self._stream(), _p(idx), _p(w), _p(counts))
         if s != LMOE_OK:
             raise LmoeError(s, "latentmoe_forward")
+        return y
+
+    def forward_block(self, x, norm_w, norm_eps=1e-5, y=None, idx=None, w=None, counts=None):
+        """y = x + layer(rmsnorm(x) * norm_w) (x bf16)."""
+        torch = self.torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.shape.H), dtype=torch.float32, device=x.device)
+        ws, n = self.workspace(T)
+        s = latentmoe_forward_block(self.h, _p(x), T, _p(norm_w), float(norm_eps), _p(y), _p(ws), ws.numel(),
+                                    self._stream(), _p(idx), _p(w), _p(counts))
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_forward_block")
         return y
 
     def route(self, x, idx=None, w=None, counts=None):

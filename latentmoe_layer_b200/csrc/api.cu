@@ -99,6 +99,7 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     p.slot = take(A * 4);
     p.wperm = take(A * 4);
     p.xbf = (c.mode == LMOE_MODE_BF16 && c.x_dtype == LMOE_FP32) ? take((size_t)T * H * 2) : 0;
+    p.xnorm = c.x_dtype == LMOE_BF16 ? take((size_t)T * H * 2) : 0;  // latentmoe_forward_block
     p.z = take((size_t)T * L * act);
     p.zperm = take(A * L * act);
     p.aperm = take(A * I * act);
@@ -319,79 +320,19 @@ __global__ void k_publish_error(const int* derr, int* herr) {
     if (v != 0) *(volatile int*)herr = v;
 }
 
-}  // namespace
-
-extern "C" {
-
-lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out) {
-    if (!out) return LMOE_ERR_INVALID_ARG;
-    lmoe_status s = check_config(cfg);
-    if (s != LMOE_OK) return s;
-    s = check_weights(w);
-    if (s != LMOE_OK) return s;
-    if (!get_encoder()) return LMOE_ERR_CUDA;
-    lmoe_handle* h = new (std::nothrow) lmoe_handle();
-    if (!h) return LMOE_ERR_INTERNAL;
-    h->cfg = *cfg;
-    h->w = *w;
-    if (cudaHostAlloc(reinterpret_cast<void**>(&h->herr), 64, cudaHostAllocMapped) != cudaSuccess) {
-        delete h;
-        return LMOE_ERR_CUDA;
-    }
-    *h->herr = 0;
-    if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->derr), h->herr, 0) != cudaSuccess) {
-        cudaFreeHost(h->herr);
-        delete h;
-        return LMOE_ERR_CUDA;
-    }
-    h->num_sms = tc_num_sms();
-    *out = h;
-    return LMOE_OK;
-}
-
-lmoe_status latentmoe_workspace_size(const lmoe_handle* h, int T, size_t* bytes) {
-    if (!h || !bytes || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
-    Plan p;
-    plan_of(h->cfg, T, p);
-    *bytes = T == 0 ? 0 : p.total;
-    return LMOE_OK;
-}
-
-lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_idx, float* topk_w,
-                            int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream) {
-    Plan p;
-    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
-    if (s != LMOE_OK || T == 0) return s;
-    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
-        (expert_counts && !aligned(expert_counts, 4)))
-        return LMOE_ERR_INVALID_ARG;
-    s = take_device_error(h);
-    if (s != LMOE_OK) return s;
-    Ctx c = make_ctx(h, p, ws, stream);
-    h->launches = 0;
-    s = do_route(c, x, topk_idx, topk_w, expert_counts);
-    if (s != LMOE_OK) return s;
-    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
-    h->launches += 1;
-    return cuda_status(cudaGetLastError());
-}
-
-lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, void* ws, size_t ws_bytes,
-                              void* stream, int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
-    Plan p;
-    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
-    if (s != LMOE_OK || T == 0) return s;
-    if (!y || !aligned(y, 16)) return LMOE_ERR_INVALID_ARG;
-    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
-        (expert_counts && !aligned(expert_counts, 4)))
-        return LMOE_ERR_INVALID_ARG;
-    s = take_device_error(h);
-    if (s != LMOE_OK) return s;
+// The layer on x (launches 1-10 of the file comment). With `resid` (bf16
+// [T, H]) the output GEMM adds it: y = resid + layer(x).
+lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y, void* ws, void* stream,
+                         int32_t* topk_idx, float* topk_w, int32_t* expert_counts, const uint16_t* resid,
+                         const uint16_t* norm_src, const uint16_t* norm_w, double norm_eps) {
+    lmoe_status s;
     const lmoe_config& cf = h->cfg;
     Ctx c = make_ctx(h, p, ws, stream);
     char* ws_c = c.ws;
     h->launches = 0;
     mark(c, 0);
+    if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
+                                                reinterpret_cast<uint16_t*>(const_cast<void*>(x)), c.s));
     s = do_route(c, x, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
     mark(c, 1);
@@ -471,11 +412,107 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
         pr.b_ptr[0] = h->w.fc2_w;
         pr.a_ptr[1] = ws_c + p.as;
         pr.b_ptr[1] = h->w.shared_down_w;
+        pr.resid = resid;
         Operand a[1][2] = {{{ws_c + p.comb, p.T}, {ws_c + p.as, p.T}}};
         Operand b[1][2] = {{{h->w.fc2_w, H}, {h->w.shared_down_w, H}}};
         LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
     }
     mark(c, 7);
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+lmoe_status check_outputs(float* y, int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
+    if (!y || !aligned(y, 16)) return LMOE_ERR_INVALID_ARG;
+    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+        (expert_counts && !aligned(expert_counts, 4)))
+        return LMOE_ERR_INVALID_ARG;
+    return LMOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, void* ws, size_t ws_bytes,
+                                         void* stream, int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    s = check_outputs(y, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    return forward_impl(h, p, x, y, ws, stream, topk_idx, topk_w, expert_counts, nullptr, nullptr, nullptr, 0.0);
+}
+
+lmoe_status latentmoe_forward_block(lmoe_handle* h, const void* x, int T, const void* norm_w,
+                                               float norm_eps, float* y, void* ws, size_t ws_bytes, void* stream,
+                                               int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    if (h->cfg.x_dtype != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
+    if (!norm_w || !aligned(norm_w, 16) || !(norm_eps >= 0.f) || isinf(norm_eps)) return LMOE_ERR_INVALID_ARG;
+    s = check_outputs(y, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    char* xn = static_cast<char*>(ws) + p.xnorm;
+    return forward_impl(h, p, xn, y, ws, stream, topk_idx, topk_w, expert_counts, static_cast<const uint16_t*>(x),
+                        static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(norm_w), (double)norm_eps);
+}
+
+
+lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out) {
+    if (!out) return LMOE_ERR_INVALID_ARG;
+    lmoe_status s = check_config(cfg);
+    if (s != LMOE_OK) return s;
+    s = check_weights(w);
+    if (s != LMOE_OK) return s;
+    if (!get_encoder()) return LMOE_ERR_CUDA;
+    lmoe_handle* h = new (std::nothrow) lmoe_handle();
+    if (!h) return LMOE_ERR_INTERNAL;
+    h->cfg = *cfg;
+    h->w = *w;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&h->herr), 64, cudaHostAllocMapped) != cudaSuccess) {
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    *h->herr = 0;
+    if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->derr), h->herr, 0) != cudaSuccess) {
+        cudaFreeHost(h->herr);
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    h->num_sms = tc_num_sms();
+    *out = h;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_workspace_size(const lmoe_handle* h, int T, size_t* bytes) {
+    if (!h || !bytes || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    Plan p;
+    plan_of(h->cfg, T, p);
+    *bytes = T == 0 ? 0 : p.total;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_idx, float* topk_w,
+                            int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+        (expert_counts && !aligned(expert_counts, 4)))
+        return LMOE_ERR_INVALID_ARG;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    Ctx c = make_ctx(h, p, ws, stream);
+    h->launches = 0;
+    s = do_route(c, x, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
     h->launches += 1;
     return cuda_status(cudaGetLastError());

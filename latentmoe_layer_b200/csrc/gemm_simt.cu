@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const GemmProblem pr, const D
             }
             if (pr.epi == EPI_SCALE_F32) v *= pr.row_scale[row];
             const long long o = row * pr.ldo + col0 + tx * 4 + j;
+            if (pr.resid) v += __uint_as_float((uint32_t)pr.resid[o] << 16);
             if (pr.epi == EPI_BF16 || pr.epi == EPI_RELU2_BF16)
                 static_cast<__nv_bfloat16*>(pr.out)[o] = __float2bfloat16_rn(v);
             else

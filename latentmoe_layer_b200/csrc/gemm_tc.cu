@@ -186,6 +186,19 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
             acc[i] = a * a;
         }
     }
+    if (!kSwap && pr.resid && lane_row < ti.rows) {  // block residual: out = resid + acc (fp32)
+        const uint4* rs = reinterpret_cast<const uint4*>(pr.resid + (size_t)(ti.row0 + lane_row) * pr.ldo + ti.col0 + c0);
+#pragma unroll
+        for (int q8 = 0; q8 < CW / 8; ++q8) {
+            const uint4 u = __ldg(rs + q8);
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[q8 * 8 + 2 * j] += __uint_as_float(w4[j] << 16);
+                acc[q8 * 8 + 2 * j + 1] += __uint_as_float(w4[j] & 0xFFFF0000u);
+            }
+        }
+    }
     if (!kSwap) {
         const bool bf16_out = epi == EPI_BF16 || epi == EPI_RELU2_BF16;
         const int slab0 = lane_row - lane;  // first row of this warp's 32-row slab
@@ -259,6 +272,7 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
                 const long long row = ti.row0 + tok;
                 float x = acc[i];
                 if (epi == EPI_SCALE_F32) x *= __ldg(&pr.row_scale[row]);
+                if (pr.resid) x += __uint_as_float((uint32_t)pr.resid[row * pr.ldo + col] << 16);
                 if (epi == EPI_BF16 || epi == EPI_RELU2_BF16)
                     static_cast<__nv_bfloat16*>(pr.out)[row * pr.ldo + col] = __float2bfloat16_rn(x);
                 else

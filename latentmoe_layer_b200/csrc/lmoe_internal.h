@@ -54,6 +54,7 @@ struct GemmProblem {
     long long ldo;          // elements
     const float* row_scale; // EPI_SCALE_F32
     int out_map;            // tensor map of `out` for bulk tensor stores (-1: plain stores)
+    const uint16_t* resid;  // EPI_F32 only: bf16 [rows, ldo] added to the result (block residual)
 };
 
 struct DeviceRouting {
@@ -69,7 +70,7 @@ struct DeviceRouting {
 struct Plan {
     size_t total;
     size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, blockcounts, perm,
-        slot, wperm, xbf, z, zperm, aperm, o, comb, as;
+        slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as;
     int T, A, nblk;
 };
 
@@ -87,6 +88,8 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* offsets_E,
                                int row_bytes, cudaStream_t s);
 cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
+                           cudaStream_t s);
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out,
                            cudaStream_t s);
 cudaError_t launch_update_bias(const int32_t* counts, const float* bias_in, int E, double eta, float* bias_out,
                                double* maxvio, cudaStream_t s);

@@ -285,6 +285,47 @@ __global__ void __launch_bounds__(1024)
     if (e == 0 && maxvio) *maxvio = mean > 0.0 ? __ddiv_rn(__dsub_rn((double)s_max[0], mean), mean) : 0.0;
 }
 
+// Nearest-even bf16 of a double (normal range): keep 8 significant bits.
+__device__ __forceinline__ double round_bf16_f64(double v) {
+    unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    u += 0x00000FFFFFFFFFFFull + ((u >> 45) & 1ull);
+    u &= ~0x00001FFFFFFFFFFFull;
+    return __longlong_as_double((long long)u);
+}
+__device__ __forceinline__ uint16_t bf16_bits(double v) { return (uint16_t)(__float_as_uint((float)v) >> 16); }
+
+// Pre-norm RMSNorm of the block ("Nemotron 3 Ultra 架构 QA", Q2.8): per token,
+// r = 1 / sqrt(mean(x^2) + eps) in fp64 (squares of bf16 are exact, sqrt and
+// division correctly rounded), xt = bf16(x r), out = bf16(gamma xt); explicit
+// round-to-nearest operations keep every rounding the same as the definition.
+__global__ void __launch_bounds__(256)
+    k_rmsnorm(const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, double eps, int T, int H,
+              uint16_t* __restrict__ out) {
+    __shared__ double red[8];
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        const uint16_t* xr = x + (size_t)t * H;
+        double ss = 0.0;
+        for (int h = threadIdx.x; h < H; h += blockDim.x) {
+            const double v = (double)__uint_as_float((uint32_t)xr[h] << 16);
+            ss = __dadd_rn(ss, __dmul_rn(v, v));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, off));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        double tot = 0.0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot = __dadd_rn(tot, red[i]);
+        __syncthreads();
+        const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(tot, (double)H), eps)));
+        for (int h = threadIdx.x; h < H; h += blockDim.x) {
+            const double v = (double)__uint_as_float((uint32_t)xr[h] << 16);
+            const double xt = round_bf16_f64(__dmul_rn(v, r));
+            const double g = (double)__uint_as_float((uint32_t)gamma[h] << 16);
+            out[(size_t)t * H + h] = bf16_bits(round_bf16_f64(__dmul_rn(g, xt)));
+        }
+    }
+}
+
 inline int grid_cap(long long work, int per_block, int cap) {
     long long g = (work + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -337,6 +378,12 @@ cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStre
     long long n4 = n / 4;
     k_convert<<<grid_cap(n4, 256, 148 * 16), 256, 0, s>>>(reinterpret_cast<const float4*>(x),
                                                           reinterpret_cast<uint2*>(xb), n4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out,
+                           cudaStream_t s) {
+    k_rmsnorm<<<T < 148 * 8 ? T : 148 * 8, 256, 0, s>>>(x, gamma, eps, T, H, out);
     return cudaGetLastError();
 }
 

@@ -57,6 +57,10 @@ def _get():
         lib.lmo_route.argtypes = [vp, vp, vp, vp, i64, vp, vp]
         lib.lmo_forward.argtypes = [vp, vp, vp, i64, vp, vp, vp]
         lib.lmo_update_bias.argtypes = [ctypes.c_int, vp, vp, ctypes.c_double, vp, vp]
+        lib.lmo_rmsnorm.argtypes = [ctypes.c_int, vp, vp, ctypes.c_double, i64, vp]
+        lib.lmo_rmsnorm.restype = ctypes.c_int
+        lib.lmo_forward_block.argtypes = [vp, vp, vp, ctypes.c_double, vp, i64, vp, vp, vp]
+        lib.lmo_forward_block.restype = ctypes.c_int
         lib.lmo_update_bias.restype = ctypes.c_int
         for f in (lib.lmo_select, lib.lmo_logits, lib.lmo_route, lib.lmo_forward):
             f.restype = ctypes.c_int
@@ -117,14 +121,7 @@ def route(cfg: LmoCfg, x, router_w, e_bias):
     return idx, w
 
 
-def forward(cfg: LmoCfg, x, wts: dict):
-    """Full layer on the rows of x. wts: router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
-    shared_up_w, shared_down_w (bf16 as uint16). up_w/down_w are [E, ...] arrays or
-    lists of per-expert arrays (None where not needed)."""
-    x = _xarr(cfg, x)
-    n = x.shape[0]
-    keep = []
-
+def _weights(cfg: LmoCfg, wts: dict, keep: list):
     def ptr(a, dt):
         a = _c(a, dt)
         keep.append(a)
@@ -138,9 +135,19 @@ def forward(cfg: LmoCfg, x, wts: dict):
         keep.append(ps)
         return ctypes.cast(ps, ctypes.c_void_p).value
 
-    W = LmoWeights(ptr(wts["router_w"], np.uint16), ptr(wts["e_bias"], np.float32), ptr(wts["fc1_w"], np.uint16),
-                   ptr(wts["fc2_w"], np.uint16), expert_ptrs(wts["up_w"]), expert_ptrs(wts["down_w"]),
-                   ptr(wts["shared_up_w"], np.uint16), ptr(wts["shared_down_w"], np.uint16))
+    return LmoWeights(ptr(wts["router_w"], np.uint16), ptr(wts["e_bias"], np.float32), ptr(wts["fc1_w"], np.uint16),
+                      ptr(wts["fc2_w"], np.uint16), expert_ptrs(wts["up_w"]), expert_ptrs(wts["down_w"]),
+                      ptr(wts["shared_up_w"], np.uint16), ptr(wts["shared_down_w"], np.uint16))
+
+
+def forward(cfg: LmoCfg, x, wts: dict):
+    """Full layer on the rows of x. wts: router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
+    shared_up_w, shared_down_w (bf16 as uint16). up_w/down_w are [E, ...] arrays or
+    lists of per-expert arrays (None where not needed)."""
+    x = _xarr(cfg, x)
+    n = x.shape[0]
+    keep = []
+    W = _weights(cfg, wts, keep)
     idx = np.zeros((n, cfg.k), dtype=np.int32)
     w = np.zeros((n, cfg.k), dtype=np.float64)
     y = np.zeros((n, cfg.H), dtype=np.float64)
@@ -148,6 +155,31 @@ def forward(cfg: LmoCfg, x, wts: dict):
                             y.ctypes.data)
     if rc != 0:
         raise ValueError("oracle forward failed (invalid configuration or missing expert weights)")
+    return y, idx, w
+
+
+def rmsnorm(x, gamma, eps):
+    x = _c(x, np.uint16)
+    g = _c(gamma, np.uint16)
+    out = np.zeros_like(x)
+    _get().lmo_rmsnorm(x.shape[1], x.ctypes.data, g.ctypes.data, float(eps), x.shape[0], out.ctypes.data)
+    return out
+
+
+def forward_block(cfg: LmoCfg, x, gamma, eps, wts: dict):
+    """y = x + layer(rmsnorm(x)) (x bf16)."""
+    x = _c(x, np.uint16)
+    g = _c(gamma, np.uint16)
+    n = x.shape[0]
+    keep = []
+    W = _weights(cfg, wts, keep)
+    idx = np.zeros((n, cfg.k), dtype=np.int32)
+    w = np.zeros((n, cfg.k), dtype=np.float64)
+    y = np.zeros((n, cfg.H), dtype=np.float64)
+    rc = _get().lmo_forward_block(ctypes.byref(cfg), x.ctypes.data, g.ctypes.data, float(eps), ctypes.byref(W), n,
+                                  idx.ctypes.data, w.ctypes.data, y.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle block forward failed")
     return y, idx, w
 
 

@@ -253,3 +253,42 @@ int lmo_update_bias(int E, const int32_t* counts, const float* bias, double eta,
     if (maxvio) *maxvio = mean > 0.0 ? ((double)mx - mean) / mean : 0.0;
     return 0;
 }
+
+static uint16_t bf16_bits_of(double v) { /* v already a bf16 value */
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* RMSNorm ("Nemotron 3 Ultra 架构 QA", Q2.8): fp64 mean of squares, r =
+ * 1/sqrt(mean + eps), bf16 rounding of x*r, then of gamma times that. */
+int lmo_rmsnorm(int H, const uint16_t* x, const uint16_t* gamma, double eps, int64_t n, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n; ++t) {
+        double ss = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double v = bf(x[t * H + h]);
+            ss += v * v;
+        }
+        const double r = 1.0 / sqrt(ss / (double)H + eps);
+        for (int h = 0; h < H; ++h) {
+            const double xt = lmo_round_bf16(bf(x[t * H + h]) * r);
+            out[t * H + h] = bf16_bits_of(lmo_round_bf16(bf(gamma[h]) * xt));
+        }
+    }
+    return 0;
+}
+
+/* Pre-norm residual block around the layer (Q2.1): y = x + layer(rmsnorm(x)). */
+int lmo_forward_block(const lmo_cfg* cfg, const uint16_t* x, const uint16_t* gamma, double eps,
+                      const lmo_weights* wts, int64_t n, int32_t* idx, double* w, double* y) {
+    if (cfg->x_f32) return -1;
+    const int H = cfg->H;
+    uint16_t* xn = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n > 0 ? n : 1) * H);
+    lmo_rmsnorm(H, x, gamma, eps, n, xn);
+    int rc = lmo_forward(cfg, xn, wts, n, idx, w, y);
+    for (int64_t i = 0; rc == 0 && i < n * H; ++i) y[i] += bf(x[i]);
+    free(xn);
+    return rc;
+}

@@ -76,6 +76,16 @@ int lmo_route(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, const
 int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64_t n, int32_t* idx, double* w,
                 double* y);
 
+/* Pre-norm RMSNorm of the block around the layer ("Nemotron 3 Ultra 架构 QA",
+ * Q2.8, the quoted forward; Q2.1: pre-norm + residual around each mixer):
+ *   r = 1 / sqrt(mean_h x[h]^2 + eps),  xt = bf16(x * r),  out = bf16(gamma * xt)
+ * x and gamma bf16, out bf16 bits; the mean and r in fp64 (the page upcasts). */
+int lmo_rmsnorm(int H, const uint16_t* x, const uint16_t* gamma, double eps, int64_t n, uint16_t* out);
+
+/* Block: y = x + layer(rmsnorm(x)) for n tokens (x bf16; y fp64 [n, H]). */
+int lmo_forward_block(const lmo_cfg* cfg, const uint16_t* x, const uint16_t* gamma, double eps,
+                      const lmo_weights* wts, int64_t n, int32_t* idx, double* w, double* y);
+
 /* Load-balancing bias update ("Nemotron 3 Ultra 架构 QA", Q5.3: the training
  * framework counts the tokens each expert received and moves the bias against
  * the overload): mean = sum(counts) / E,

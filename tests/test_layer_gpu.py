@@ -12,6 +12,7 @@ import pytest
 import synth
 from synth import LayerShape, TINY, NANO_DECODE, ULTRA_DECODE, ULTRA_PREFILL, ULTRA_SKEW
 import helpers as H
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -195,3 +196,27 @@ def test_near_edge_recheck_margin():
         if name != "none":
             assert mism == 0
     assert flagged["wide"] > 0 and flagged["none"] == 0
+
+
+def _gamma(H):
+    import torch
+    g = torch.from_numpy(np.random.default_rng(11).uniform(0.5, 1.5, H).astype(np.float32)).to(torch.bfloat16)
+    return g.cuda()
+
+
+@pytest.mark.parametrize("shape,path", [(RAGGED, GEMM_PREFILL), (RAGGED, GEMM_DECODE), (NANO_DECODE, GEMM_AUTO)])
+def test_pre_norm_residual_block(shape, path):
+    """y = x + layer(rmsnorm(x)): routing of the normed input bit-exact, y within tolerance."""
+    import torch
+    layer, dev = H.device_layer(shape)
+    layer.set_option(0, path)
+    g = _gamma(shape.H)
+    T = shape.T
+    idx = torch.empty((T, shape.k), dtype=torch.int32, device="cuda")
+    y = layer.forward_block(dev["x"], g, 1e-5, idx=idx)
+    torch.cuda.synchronize()
+    host = synth.host_inputs(shape)
+    yref, iref, _ = oracle.forward_block(oracle.make_cfg(shape), host["x"], H.bf16_to_bits(g), 1e-5, host)
+    assert np.array_equal(idx.cpu().numpy(), iref)
+    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref, wide=H.is_wide(shape))
+    print("block %s path=%d max_abs=%.3g rel_fro=%.3g" % (shape.name, path, ma, rf))

@@ -374,3 +374,43 @@ def test_bias_update_moves_against_overload(built_oracle):
 def test_bias_update_empty_batch(built_oracle):
     nb, mv = built_oracle.update_bias(np.zeros(8, np.int32), np.ones(8, np.float32), 0.5)
     assert np.array_equal(nb, np.ones(8, np.float32)) and mv == 0.0
+
+
+# ------------------------------------------------------------------ pre-norm RMSNorm block (Q2.8, Q2.1)
+def test_rmsnorm_is_a_correct_rounding_of_torch_rms_norm(built_oracle):
+    rng = np.random.default_rng(4)
+    H = 512
+    x = f32_to_bf16_bits(rng.standard_normal((6, H)).astype(np.float32) * 3.0)
+    ones = f32_to_bf16_bits(np.ones(H, np.float32))
+    out = bits_to_f64(built_oracle.rmsnorm(x, ones, 1e-5))
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(bits_to_f64(x)), (H,), eps=1e-5).numpy()
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(ref))[1] - 9)   # half a bf16 ulp of each reference value
+    assert np.all(np.abs(out - ref) <= half_ulp * (1 + 1e-9))
+
+
+def test_rmsnorm_closed_forms(built_oracle):
+    H = 64
+    sign = np.where(np.arange(H) % 3 == 0, -1.0, 1.0).astype(np.float32)
+    x = f32_to_bf16_bits(2.0 * sign[None, :])
+    # |x| = 2 everywhere: r = 1/sqrt(4 + eps) and bf16(x r) = +-1; gamma = 1.5 gives +-1.5
+    g = f32_to_bf16_bits(np.full(H, 1.5, np.float32))
+    assert np.array_equal(bits_to_f64(built_oracle.rmsnorm(x, g, 1e-5)), 1.5 * sign[None, :])
+    # without eps the norm is invariant to scaling x by a power of two
+    rng = np.random.default_rng(5)
+    xr = f32_to_bf16_bits(rng.standard_normal((3, H)).astype(np.float32))
+    g = f32_to_bf16_bits(rng.uniform(0.5, 1.5, H).astype(np.float32))
+    a = built_oracle.rmsnorm(xr, g, 0.0)
+    b = built_oracle.rmsnorm(f32_to_bf16_bits(bits_to_f64(xr).astype(np.float32) * 8.0), g, 0.0)
+    assert np.array_equal(a, b)
+
+
+def test_block_is_residual_plus_layer_of_normed_input(built_oracle):
+    w = small_shape(E=8, k=2, T=5, x_f32=False)
+    cfg = built_oracle.make_cfg(w)
+    inp = inputs(w)
+    g = f32_to_bf16_bits(np.random.default_rng(6).uniform(0.5, 1.5, w.H).astype(np.float32))
+    y, idx, _ = built_oracle.forward_block(cfg, inp["x"], g, 1e-5, inp)
+    xn = built_oracle.rmsnorm(inp["x"], g, 1e-5)
+    y2, idx2, _ = built_oracle.forward(cfg, xn, inp)
+    assert np.array_equal(idx, idx2)
+    assert np.array_equal(y, y2 + bits_to_f64(inp["x"]))
