@@ -31,7 +31,8 @@ class LmoCfg(ctypes.Structure):
 class LmoWeights(ctypes.Structure):
     _fields_ = [("router_w", ctypes.c_void_p), ("e_bias", ctypes.c_void_p), ("fc1_w", ctypes.c_void_p),
                 ("fc2_w", ctypes.c_void_p), ("up_w", ctypes.c_void_p), ("down_w", ctypes.c_void_p),
-                ("shared_up_w", ctypes.c_void_p), ("shared_down_w", ctypes.c_void_p)]
+                ("shared_up_w", ctypes.c_void_p), ("shared_down_w", ctypes.c_void_p),
+                ("up_gs", ctypes.c_void_p), ("down_gs", ctypes.c_void_p)]
 
 
 def build(force: bool = False):
@@ -62,6 +63,18 @@ def _get():
         lib.lmo_forward_block.argtypes = [vp, vp, vp, ctypes.c_double, vp, i64, vp, vp, vp]
         lib.lmo_forward_block.restype = ctypes.c_int
         lib.lmo_update_bias.restype = ctypes.c_int
+        lib.lmo_e2m1_value.argtypes = [ctypes.c_int]
+        lib.lmo_e2m1_value.restype = ctypes.c_double
+        lib.lmo_e4m3_value.argtypes = [ctypes.c_int]
+        lib.lmo_e4m3_value.restype = ctypes.c_double
+        lib.lmo_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.lmo_e2m1_encode.restype = ctypes.c_int
+        lib.lmo_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.lmo_e4m3_encode.restype = ctypes.c_int
+        lib.lmo_nvfp4_quantize.argtypes = [vp, i64, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+        lib.lmo_nvfp4_quantize.restype = ctypes.c_int
+        lib.lmo_nvfp4_dequant.argtypes = [vp, vp, i64, ctypes.c_int, ctypes.c_int, vp]
+        lib.lmo_nvfp4_dequant.restype = ctypes.c_int
         for f in (lib.lmo_select, lib.lmo_logits, lib.lmo_route, lib.lmo_forward):
             f.restype = ctypes.c_int
         _lib = lib
@@ -135,15 +148,22 @@ def _weights(cfg: LmoCfg, wts: dict, keep: list):
         keep.append(ps)
         return ctypes.cast(ps, ctypes.c_void_p).value
 
+    def opt_scales(key):
+        g = wts.get(key)
+        return None if g is None else ptr(np.asarray(g, dtype=np.float32), np.float32)
+
     return LmoWeights(ptr(wts["router_w"], np.uint16), ptr(wts["e_bias"], np.float32), ptr(wts["fc1_w"], np.uint16),
                       ptr(wts["fc2_w"], np.uint16), expert_ptrs(wts["up_w"]), expert_ptrs(wts["down_w"]),
-                      ptr(wts["shared_up_w"], np.uint16), ptr(wts["shared_down_w"], np.uint16))
+                      ptr(wts["shared_up_w"], np.uint16), ptr(wts["shared_down_w"], np.uint16),
+                      opt_scales("up_gs"), opt_scales("down_gs"))
 
 
 def forward(cfg: LmoCfg, x, wts: dict):
     """Full layer on the rows of x. wts: router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
     shared_up_w, shared_down_w (bf16 as uint16). up_w/down_w are [E, ...] arrays or
-    lists of per-expert arrays (None where not needed)."""
+    lists of per-expert arrays (None where not needed). Optional up_gs / down_gs
+    ([E] fp32): per-expert matrix scales of NVFP4 experts (up_w/down_w then hold
+    the dequantised code * block-scale values, see nvfp4_dequant)."""
     x = _xarr(cfg, x)
     n = x.shape[0]
     keep = []
@@ -192,3 +212,45 @@ def update_bias(counts, bias, eta):
     _get().lmo_update_bias(len(bias), counts.ctypes.data, bias.ctypes.data, float(eta), out.ctypes.data,
                            ctypes.byref(mv))
     return out, mv.value
+
+
+# ---------------------------------------------------------------- NVFP4
+def e2m1_value(code: int) -> float:
+    return _get().lmo_e2m1_value(int(code))
+
+
+def e4m3_value(byte: int) -> float:
+    return _get().lmo_e4m3_value(int(byte))
+
+
+def e2m1_encode(q: float) -> int:
+    return _get().lmo_e2m1_encode(float(q))
+
+
+def e4m3_encode(u: float) -> int:
+    return _get().lmo_e4m3_encode(float(u))
+
+
+def nvfp4_quantize(w):
+    """w: [n_mat, R, K] bf16 bits (uint16). Returns (codes uint8 [n_mat*R*K/2],
+    sf uint8 [n_mat*R*K/16], g float32 [n_mat]) in the tiled layout of oracle.h."""
+    w = _c(w, np.uint16)
+    n_mat, R, K = w.shape
+    codes = np.zeros(n_mat * R * K // 2, dtype=np.uint8)
+    sf = np.zeros(n_mat * R * K // 16, dtype=np.uint8)
+    g = np.zeros(n_mat, dtype=np.float32)
+    rc = _get().lmo_nvfp4_quantize(w.ctypes.data, n_mat, R, K, codes.ctypes.data, sf.ctypes.data, g.ctypes.data)
+    if rc != 0:
+        raise ValueError("NVFP4 quantisation needs R % 128 == 0 and K % 64 == 0")
+    return codes, sf, g
+
+
+def nvfp4_dequant(codes, sf, n_mat, R, K):
+    """bf16 bits [n_mat, R, K] of code_value * block scale (the matrix scale g not applied)."""
+    codes = _c(codes, np.uint8)
+    sf = _c(sf, np.uint8)
+    out = np.zeros((n_mat, R, K), dtype=np.uint16)
+    rc = _get().lmo_nvfp4_dequant(codes.ctypes.data, sf.ctypes.data, n_mat, R, K, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("NVFP4 dequantisation: bad shape or inexact product")
+    return out

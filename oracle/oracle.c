@@ -207,16 +207,19 @@ int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64
                 bad = 1;
                 break;
             }
+            const double gu = wts->up_gs ? (double)wts->up_gs[idx[j]] : 1.0;
+            const double gd = wts->down_gs ? (double)wts->down_gs[idx[j]] : 1.0;
             for (int i = 0; i < I; ++i) {
                 double s = 0.0;
                 for (int l = 0; l < L; ++l) s += z[l] * bf(up[(int64_t)i * L + l]);
+                s *= gu;
                 double r = s > 0.0 ? s : 0.0;
                 a[i] = rho(cfg, r * r);
             }
             for (int l = 0; l < L; ++l) {
                 double s = 0.0;
                 for (int i = 0; i < I; ++i) s += a[i] * bf(dn[(int64_t)l * I + i]);
-                acc[l] += w[j] * s;
+                acc[l] += w[j] * (gd * s);
             }
         }
         for (int l = 0; l < L; ++l) comb[l] = rho(cfg, acc[l]);
@@ -291,4 +294,110 @@ int lmo_forward_block(const lmo_cfg* cfg, const uint16_t* x, const uint16_t* gam
     for (int64_t i = 0; rc == 0 && i < n * H; ++i) y[i] += bf(x[i]);
     free(xn);
     return rc;
+}
+
+/* ---------------------------------------------------------------- NVFP4
+ * Format and recipe as stated in oracle.h. Decoding follows the bit fields;
+ * encoding is a brute-force search over every representable value, so no
+ * bit trick of the encoder needs checking. */
+double lmo_e2m1_value(int code) {
+    const int e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+double lmo_e4m3_value(int byte) {
+    const int e = (byte >> 3) & 15, m = byte & 7;
+    if ((byte & 0x7F) == 0x7F) return NAN;
+    const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (byte & 0x80) ? -mag : mag;
+}
+
+/* nearest of the candidate codes lo..hi (non-negative values, ascending), ties to the even code */
+static int nearest_code(double a, int hi, double (*val)(int)) {
+    int best = 0;
+    double bd = fabs(val(0) - a);
+    for (int c = 1; c <= hi; ++c) {
+        const double d = fabs(val(c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return best;
+}
+
+int lmo_e2m1_encode(float q) {
+    const int s = q < 0.0f;
+    const double a = fabs((double)q);
+    const int m = a >= 6.0 ? 7 : nearest_code(a, 7, lmo_e2m1_value);
+    return (s << 3) | m;
+}
+
+int lmo_e4m3_encode(float u) {
+    if (!(u > 0.0f)) return 0;
+    if ((double)u >= 448.0) return 0x7E;
+    return nearest_code((double)u, 0x7E, lmo_e4m3_value);
+}
+
+static inline int64_t tile_of(int64_t gr, int K, int k) { return (gr / 128) * (K / 64) + k / 64; }
+
+int lmo_nvfp4_quantize(const uint16_t* w, int64_t n_mat, int R, int K, uint8_t* codes, uint8_t* sf, float* g) {
+    if (R <= 0 || K <= 0 || R % 128 || K % 64) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < n_mat; ++m) {
+        const uint16_t* wm = w + m * (int64_t)R * K;
+        float amax = 0.0f;
+        for (int64_t i = 0; i < (int64_t)R * K; ++i) {
+            const float a = fabsf((float)bf(wm[i]));
+            if (a > amax) amax = a;
+        }
+        const float gm = amax > 0.0f ? amax / 2688.0f : 1.0f;
+        g[m] = gm;
+        for (int r = 0; r < R; ++r) {
+            const int64_t gr = m * R + r;
+            for (int b = 0; b < K / 16; ++b) {
+                const int k0 = b * 16;
+                float bmax = 0.0f;
+                for (int i = 0; i < 16; ++i) {
+                    const float a = fabsf((float)bf(wm[(int64_t)r * K + k0 + i]));
+                    if (a > bmax) bmax = a;
+                }
+                const float t = bmax / gm;
+                const float u = t / 6.0f;
+                const int sb = lmo_e4m3_encode(u);
+                const float S = (float)lmo_e4m3_value(sb);
+                sf[tile_of(gr, K, k0) * 512 + (gr % 128) * 4 + (k0 % 64) / 16] = (uint8_t)sb;
+                const float d = S * gm;
+                for (int i = 0; i < 16; i += 2) {
+                    int c[2];
+                    for (int h = 0; h < 2; ++h) {
+                        const float wv = (float)bf(wm[(int64_t)r * K + k0 + i + h]);
+                        c[h] = S == 0.0f ? 0 : lmo_e2m1_encode(wv / d);
+                    }
+                    const int k = k0 + i;
+                    codes[tile_of(gr, K, k) * 4096 + (gr % 128) * 32 + (k % 64) / 2] = (uint8_t)(c[0] | (c[1] << 4));
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+int lmo_nvfp4_dequant(const uint8_t* codes, const uint8_t* sf, int64_t n_mat, int R, int K, uint16_t* out) {
+    if (R <= 0 || K <= 0 || R % 128 || K % 64) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t gr = 0; gr < n_mat * R; ++gr) {
+        for (int k = 0; k < K; ++k) {
+            const int64_t t = tile_of(gr, K, k);
+            const uint8_t byte = codes[t * 4096 + (gr % 128) * 32 + (k % 64) / 2];
+            const int code = (k & 1) ? byte >> 4 : byte & 15;
+            const double S = lmo_e4m3_value(sf[t * 512 + (gr % 128) * 4 + (k % 64) / 16]);
+            const double v = lmo_e2m1_value(code) * S;
+            if (lmo_round_bf16(v) != v) bad = 1; /* code * S always has <= 6 significant bits */
+            out[gr * K + k] = bf16_bits_of(v);
+        }
+    }
+    return bad ? -1 : 0;
 }

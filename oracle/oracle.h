@@ -54,6 +54,11 @@ typedef struct {
     const uint16_t* const* down_w; /* E pointers, each [L, I]; NULL where unused */
     const uint16_t* shared_up_w;   /* [Is, H] */
     const uint16_t* shared_down_w; /* [H, Is] */
+    /* Per-expert matrix scales of block-scaled (NVFP4) experts, or NULL (1.0):
+     * h = up_gs[e] * (z . W_up[e] row), o = w * down_gs[e] * (a . W_down[e] row),
+     * the scale applied to the accumulated product before the activation. */
+    const float* up_gs;            /* [E] or NULL */
+    const float* down_gs;          /* [E] or NULL */
 } lmo_weights;
 
 #define LMO_EPS 1e-6
@@ -94,6 +99,38 @@ int lmo_forward_block(const lmo_cfg* cfg, const uint16_t* x, const uint16_t* gam
  *   = (max_e counts[e] - mean) / mean   (0 when no token was routed).
  * bias_out may alias bias. Returns 0. */
 int lmo_update_bias(int E, const int32_t* counts, const float* bias, double eta, float* bias_out, double* maxvio);
+
+/* ---- NVFP4 block-scaled expert weights ("Nemotron 3 Ultra 架构 QA", Q1.3 and
+ * Q8.1: the 512 experts' up and down weights are the layers kept in NVFP4, the
+ * latent projections fc1/fc2 stay BF16; overview page: NVFP4 quantisation for
+ * inference). The pages name the format but do not spell it out; this is its
+ * public definition:
+ *   element  E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa;
+ *            magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6
+ *   block    16 consecutive elements along K share one E4M3 scale S (finite
+ *            variant: bias 7, 3 mantissa bits, subnormals, max 448, no inf)
+ *   matrix   one fp32 scale g per matrix (per expert and projection)
+ *   value    w = code_value * S * g
+ * Quantisation (reading of the usual recipe, all decisions in fp32 with
+ * round-to-nearest-even operations):
+ *   amax = max |w| of the matrix;  g = amax / 2688 (6 * 448), or 1 if amax = 0
+ *   per block: S = E4M3 nearest to (bmax / g) / 6, saturating at 448
+ *   per element: q = w / (S * g) (product rounded to fp32 first);
+ *                code = E2M1 nearest to q, ties to the even mantissa,
+ *                saturating at 6; sign bit = (q < 0); S = 0 gives code 0.
+ * Storage (tiles of 128 rows x 64 K; R multiple of 128, K multiple of 64):
+ *   global row gr = m * R + r, tile id = (gr / 128) * (K / 64) + k / 64
+ *   codes: byte tile*4096 + (gr % 128)*32 + (k % 64)/2, even k in the low nibble
+ *   scales: byte tile*512 + (gr % 128)*4 + (k % 64)/16                      */
+double lmo_e2m1_value(int code);
+double lmo_e4m3_value(int byte);            /* NaN for 0x7F / 0xFF */
+int lmo_e2m1_encode(float q);               /* nearest code, ties to even, saturating */
+int lmo_e4m3_encode(float u);               /* u >= 0: nearest, ties to even, saturating */
+/* n_mat matrices of [R, K] bf16 -> codes, scales (tiled layout) and g[n_mat].
+ * Returns 0, or -1 when R % 128 or K % 64 is non-zero. */
+int lmo_nvfp4_quantize(const uint16_t* w, int64_t n_mat, int R, int K, uint8_t* codes, uint8_t* sf, float* g);
+/* bf16 bits of code_value * S (exact) for the n_mat x R x K elements (g not applied). */
+int lmo_nvfp4_dequant(const uint8_t* codes, const uint8_t* sf, int64_t n_mat, int R, int K, uint16_t* out);
 
 #ifdef __cplusplus
 }

@@ -414,3 +414,156 @@ def test_block_is_residual_plus_layer_of_normed_input(built_oracle):
     y2, idx2, _ = built_oracle.forward(cfg, xn, inp)
     assert np.array_equal(idx, idx2)
     assert np.array_equal(y, y2 + bits_to_f64(inp["x"]))
+
+
+# ---------------------------------------------------------------- NVFP4 experts
+E2M1_MAGNITUDES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_follows_bit_fields(built_oracle):
+    got = [built_oracle.e2m1_value(c) for c in range(16)]
+    assert got[:8] == E2M1_MAGNITUDES
+    assert got[8:] == [-v for v in E2M1_MAGNITUDES]
+
+
+def test_e4m3_decode_matches_torch_float8(built_oracle):
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([built_oracle.e4m3_value(b) for b in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got)) and nan.sum() == 2
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert built_oracle.e4m3_value(0x7E) == 448.0 and built_oracle.e4m3_value(1) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_rounding(built_oracle):
+    rng = np.random.default_rng(11)
+    finite = [built_oracle.e4m3_value(b) for b in range(0x7F)]
+    mids = [(a + b) / 2 for a, b in zip(finite[:-1], finite[1:])]      # exact ties
+    us = np.concatenate([rng.uniform(0, 448, 4000), np.exp(rng.uniform(-12, 6, 4000)), finite, mids]).astype(np.float32)
+    us = us[us <= 448]
+    ref = torch.from_numpy(us).to(torch.float8_e4m3fn).view(torch.uint8).numpy().astype(int)
+    got = np.array([built_oracle.e4m3_encode(float(u)) for u in us])
+    assert np.array_equal(ref, got)
+    assert built_oracle.e4m3_encode(1e6) == 0x7E and built_oracle.e4m3_encode(0.0) == 0
+
+
+def test_e2m1_encode_nearest_with_even_ties(built_oracle):
+    # exact midpoints go to the even mantissa (code & 1 == 0)
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    for q, c in ties.items():
+        assert built_oracle.e2m1_encode(q) == c
+        assert built_oracle.e2m1_encode(-q) == (c | 8)
+    rng = np.random.default_rng(12)
+    for q in rng.uniform(-8, 8, 3000).astype(np.float32):
+        c = built_oracle.e2m1_encode(float(q))
+        mag = E2M1_MAGNITUDES[c & 7]
+        best = min(abs(abs(q) - m) for m in E2M1_MAGNITUDES) if abs(q) < 6 else abs(q) - 6.0
+        assert abs(abs(q) - mag) == pytest.approx(best, abs=0) or (abs(q) >= 6 and c & 7 == 7)
+        assert (c >> 3) == (q < 0)
+
+
+def read_nvfp4_example():
+    scales, elems, g = {}, {}, None
+    with open(os.path.join(GOLDEN, "nvfp4_worked_example.txt"), encoding="utf-8") as f:
+        for line in f:
+            p = line.split()
+            if not p or p[0].startswith("#"):
+                continue
+            if p[0] == "g":
+                g = float(p[1])
+            elif p[0] == "scale":
+                scales[int(p[1])] = int(p[2], 16)
+            elif p[0] == "elem":
+                elems[int(p[1])] = (float(p[2]), int(p[3]))
+    return g, scales, elems
+
+
+def test_nvfp4_quantize_worked_example(built_oracle):
+    g_ref, scales, elems = read_nvfp4_example()
+    R, K, row = 128, 64, 5
+    wf = np.zeros((1, R, K), dtype=np.float32)
+    for k, (v, _) in elems.items():
+        wf[0, row, k] = v
+    w = f32_to_bf16_bits(wf).reshape(1, R, K)
+    assert np.array_equal(bits_to_f64(w).reshape(1, R, K)[0, row], wf[0, row].astype(np.float64))  # values exact
+    codes, sf, g = built_oracle.nvfp4_quantize(w)
+    assert g[0] == np.float32(g_ref)
+    for b, byte in scales.items():
+        assert sf[row * 4 + b] == byte, b
+    for k in range(K):
+        byte = codes[row * 32 + k // 2]
+        code = (byte >> 4) if k & 1 else (byte & 15)
+        assert code == elems.get(k, (0.0, 0))[1], k
+    other = np.ones(R, dtype=bool)
+    other[row] = False
+    assert not codes.reshape(R, 32)[other].any() and not sf.reshape(R, 4)[other].any()
+
+
+def nvfp4_weights(rng, n_mat, R, K, std=0.02):
+    return f32_to_bf16_bits(rng.normal(0, std, (n_mat, R, K)).astype(np.float32)).reshape(n_mat, R, K)
+
+
+def test_nvfp4_error_bound_and_block_max(built_oracle):
+    rng = np.random.default_rng(13)
+    n_mat, R, K = 2, 128, 128
+    w = nvfp4_weights(rng, n_mat, R, K)
+    codes, sf, g = built_oracle.nvfp4_quantize(w)
+    deq = bits_to_f64(built_oracle.nvfp4_dequant(codes, sf, n_mat, R, K)).reshape(n_mat, R, K)
+    wf = bits_to_f64(w).reshape(n_mat, R, K)
+    blocks = wf.reshape(n_mat, R, K // 16, 16)
+    S = np.abs(deq.reshape(n_mat, R, K // 16, 16)).max(axis=3) / 6.0  # block max element decodes to 6 * S
+    for m in range(n_mat):
+        # block scale: S = E4M3(bmax / g / 6) within half an E4M3 step (relative 1/16)
+        u = np.abs(blocks[m]).max(axis=2) / g[m] / 6.0
+        assert np.all(np.abs(S[m] - u) <= u / 16 + 1e-30)
+        d = S[m][..., None] * g[m]
+        q = blocks[m] / d
+        v = deq[m].reshape(R, K // 16, 16) * g[m]
+        # per element: error at most half the E2M1 spacing at |q| (0.5 below 2, 1 below 4, 2 above), or the
+        # saturation error above 6
+        half = np.where(np.abs(q) < 2, 0.25, np.where(np.abs(q) < 4, 0.5, 1.0)) * d
+        sat = np.maximum(np.abs(blocks[m]) - 6 * d, 0)
+        assert np.all(np.abs(blocks[m] - v) <= np.maximum(half, sat) * (1 + 1e-6))
+
+
+def test_nvfp4_requantising_the_dequantised_matrix_is_idempotent(built_oracle):
+    rng = np.random.default_rng(14)
+    n_mat, R, K = 2, 128, 64
+    codes, sf, g = built_oracle.nvfp4_quantize(nvfp4_weights(rng, n_mat, R, K))
+    deq = built_oracle.nvfp4_dequant(codes, sf, n_mat, R, K)
+    codes2, sf2, g2 = built_oracle.nvfp4_quantize(deq)
+    # the matrix maximum sits in a block with S = 448 and code 6, so g' = 6 * 448 / 2688 = 1
+    assert np.all(g2 == 1.0)
+
+    def plus_zero(c):  # -0 (code 8) dequantises to -0.0, which quantises to +0
+        lo, hi = c & 15, c >> 4
+        return np.where(lo == 8, 0, lo) | (np.where(hi == 8, 0, hi) << 4)
+
+    assert np.array_equal(sf, sf2) and np.array_equal(plus_zero(codes), plus_zero(codes2))
+    assert np.array_equal(codes2, plus_zero(codes2))
+
+
+def test_nvfp4_rejects_untiled_shapes(built_oracle):
+    with pytest.raises(ValueError):
+        built_oracle.nvfp4_quantize(np.zeros((1, 64, 64), dtype=np.uint16))
+
+
+def test_expert_matrix_scales_enter_before_the_activation(built_oracle):
+    # A power-of-two matrix scale is exact in bf16 and fp64: scaling the weights by it or passing it as
+    # the per-expert matrix scale must give bitwise the same layer (relu2 of 2h is 4 relu2(h), so a scale
+    # applied after the activation would not).
+    w = small_shape(E=8, k=3, T=6, x_f32=False)
+    cfg = built_oracle.make_cfg(w)
+    inp = inputs(w)
+    up = bits_to_f64(inp["up_w"]).astype(np.float32)
+    dn = bits_to_f64(inp["down_w"]).astype(np.float32)
+    gu = np.array([2.0 ** (e % 3) for e in range(w.E)], dtype=np.float32)
+    gd = np.array([2.0 ** -(e % 2) for e in range(w.E)], dtype=np.float32)
+    scaled = dict(inp)
+    scaled["up_w"] = f32_to_bf16_bits(up * gu[:, None, None]).reshape(inp["up_w"].shape)
+    scaled["down_w"] = f32_to_bf16_bits(dn * gd[:, None, None]).reshape(inp["down_w"].shape)
+    y1, idx1, _ = built_oracle.forward(cfg, inp["x"], dict(inp, up_gs=gu, down_gs=gd))
+    y2, idx2, _ = built_oracle.forward(cfg, inp["x"], scaled)
+    assert np.array_equal(idx1, idx2) and np.array_equal(y1, y2)
+    y3, _, _ = built_oracle.forward(cfg, inp["x"], inp)
+    assert not np.array_equal(y1, y3)
