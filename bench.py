@@ -101,11 +101,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ work accounting
-def expert_gemm_work(w, distinct):
+def expert_gemm_work(w, distinct, nvfp4=False):
     """Algorithmic FLOPs and bytes of one expert GEMM launch (up or down)."""
     A = w.T * w.k
     flops = 2.0 * A * w.L * w.I
-    weight_bytes = 2.0 * distinct * w.L * w.I
+    weight_bytes = distinct * w.L * w.I * ((0.5 + 1.0 / 16) if nvfp4 else 2.0)
     act_bytes = 2.0 * A * w.L + 2.0 * A * w.I   # bf16 operand rows in, bf16 rows out (up) / fp32 out (down ~ same order)
     return flops, weight_bytes + act_bytes
 
@@ -134,7 +134,7 @@ def dist_setup():
 
 
 # ------------------------------------------------------------------ our arm
-def measure(shape, steps, warmup, world, rank, local, dist, torch):
+def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
     import latentmoe_layer_b200 as lm
     import synth
 
@@ -151,7 +151,14 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch):
             lib.synth_cuda_fill_normal_bf16(dev["x"].data_ptr(), n, 0, synth.TID_X, 1.0, off, stream)
         if shape.skew_hot:
             dev["x"][:, 0] = 1.0
-    layer = lm.LatentMoE(shape, dev, shape.T, x_f32=shape.x_f32)
+    if nvfp4:  # expert weights converted once, before any timing
+        q = {}
+        q["up_w"], q["up_sf"], q["up_gs"] = lm.quantize_nvfp4(dev["up_w"])
+        q["down_w"], q["down_sf"], q["down_gs"] = lm.quantize_nvfp4(dev["down_w"])
+        layer = lm.LatentMoE(shape, dict(dev, **q), shape.T, x_f32=shape.x_f32, expert_format=lm.LMOE_EXPERTS_NVFP4)
+        dev["nvfp4"] = q
+    else:
+        layer = lm.LatentMoE(shape, dev, shape.T, x_f32=shape.x_f32)
     x = dev["x"]
     y = torch.empty((shape.T, shape.H), dtype=torch.float32, device="cuda")
     layer.workspace(shape.T)
@@ -254,9 +261,9 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch):
 UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT = (1.545e9 + 0.456e9) / 45056
 
 
-def roofline_for(shape, res, peaks, peak_src, prefill: bool):
+def roofline_for(shape, res, peaks, peak_src, prefill: bool, nvfp4=False):
     st = res["stats"]
-    flops, byts = expert_gemm_work(shape, st.distinct_experts)
+    flops, byts = expert_gemm_work(shape, st.distinct_experts, nvfp4)
     up_ms, dn_ms = res["stage_ms"]["expert_up_gemm"], res["stage_ms"]["expert_down_gemm"]
     name, kms = ("expert_up_gemm", up_ms) if up_ms >= dn_ms else ("expert_down_gemm", dn_ms)
     if prefill:
@@ -276,13 +283,13 @@ def roofline_for(shape, res, peaks, peak_src, prefill: bool):
             "algorithmic_per_launch": byts, "launch_ms": round(kms, 4)}
 
 
-def layer_summary(shape, res, peaks, peak_src, steps):
+def layer_summary(shape, res, peaks, peak_src, steps, nvfp4=False):
     import latentmoe_layer_b200.accounting as acc
     st = res["stats"]
     ms_step = res["ms"] / steps
     tok_s = shape.T / (ms_step * 1e-3)
     layer_flops = acc.flops_per_token(shape) * shape.T
-    layer_bytes = acc.min_bytes_per_call(shape, st.distinct_experts)
+    layer_bytes = acc.min_bytes_per_call(shape, st.distinct_experts, nvfp4)
     return {
         "ms_per_step": round(ms_step, 4), "tokens_per_s": round(tok_s, 1),
         "layer_tflops": round(layer_flops / (ms_step * 1e-3) / 1e12, 1),
@@ -348,11 +355,12 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     shape = synth.WORKLOADS[args.workload]
     prefill = shape.T * shape.k > 64 * shape.E
-    res = measure(shape, args.steps, args.warmup, world, rank, local, dist, torch)
+    nv = args.experts == "nvfp4"
+    res = measure(shape, args.steps, args.warmup, world, rank, local, dist, torch, nvfp4=nv)
     ms_step = res["ms"] / args.steps
     value = world * shape.T / (ms_step * 1e-3)
     e2e_value = world * shape.T * res["e2e_steps"] / (res["e2e_ms"] * 1e-3)
-    summary = layer_summary(shape, res, peaks, peak_src, args.steps)
+    summary = layer_summary(shape, res, peaks, peak_src, args.steps, nvfp4=nv)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -360,10 +368,11 @@ def run_ours(args):
         "config": {"workload": shape.name, "T": shape.T, "H": shape.H, "L": shape.L, "E": shape.E, "k": shape.k,
                    "n_group": shape.G, "topk_group": shape.Gk, "I": shape.I, "Is": shape.Is,
                    "global_batch": shape.T * world, "parallelism": "replicas" if world > 1 else "single",
+                   "experts": args.experts,
                    "l2": "inputs larger than L2 (%.1f GB of weights), no flush" %
                          (2 * (shape.E * 2 * shape.L * shape.I + shape.E * shape.H + 2 * shape.H * shape.L +
                                2 * shape.H * shape.Is) / 1e9)},
-        "roofline": roofline_for(shape, res, peaks, peak_src, prefill),
+        "roofline": roofline_for(shape, res, peaks, peak_src, prefill, nvfp4=nv),
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": res["stats"].kernel_launches * args.steps,
@@ -371,7 +380,7 @@ def run_ours(args):
         "layer": summary,
     }
     layer, dev = res["layer"], res["dev"]
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not nv:
         cb, _ = cpu_baseline(shape, dev)
         line["cpu_baseline"] = cb
     layer.close()
@@ -386,6 +395,19 @@ def run_ours(args):
                              "layer": layer_summary(s2, r2, peaks, peak_src, args.secondary_steps),
                              "clocks": r2["clocks"]}
         r2["layer"].close()
+        del r2
+        torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and args.nvfp4_workload not in ("", "none"):
+        # the same layer with NVFP4 routed-expert weights (dense weights stay bf16)
+        s3 = synth.WORKLOADS[args.nvfp4_workload]
+        r3 = measure(s3, args.secondary_steps, args.warmup, 1, 0, local, None, torch, nvfp4=True)
+        line["nvfp4_experts"] = {
+            "workload": s3.name, "value": round(s3.T / (r3["ms"] / args.secondary_steps * 1e-3), 1),
+            "unit": "tokens/s", "steps": args.secondary_steps,
+            "roofline": roofline_for(s3, r3, peaks, peak_src, s3.T * s3.k > 64 * s3.E, nvfp4=True),
+            "layer": layer_summary(s3, r3, peaks, peak_src, args.secondary_steps, nvfp4=True),
+            "clocks": r3["clocks"]}
+        r3["layer"].close()
     if rank == 0:
         print(json.dumps(line))
     if dist is not None:
@@ -456,6 +478,10 @@ def main():
     ap.add_argument("--workload", default="ultra_prefill")
     ap.add_argument("--secondary", default="ultra_decode", help="second workload reported under 'secondary'")
     ap.add_argument("--secondary-steps", type=int, default=200)
+    ap.add_argument("--experts", choices=["bf16", "nvfp4"], default="bf16",
+                    help="routed-expert weight format of the main measurement")
+    ap.add_argument("--nvfp4-workload", default="ultra_decode",
+                    help="workload measured again with NVFP4 expert weights ('none' to skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens-per-core", type=int, default=2)
     args = ap.parse_args()

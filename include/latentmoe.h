@@ -61,6 +61,11 @@ typedef enum {
 
 typedef enum { LMOE_BF16 = 0, LMOE_FP32 = 1 } lmoe_dtype;
 typedef enum { LMOE_MODE_BF16 = 0, LMOE_MODE_FP32 = 1 } lmoe_mode;
+/* Storage of the routed experts' up/down weights. NVFP4 ("Nemotron 3 Ultra 架构
+ * QA", Q1.3 and Q8.1: the experts' up and down projections are the NVFP4
+ * layers, the latent projections, router and shared expert stay BF16): see
+ * latentmoe_quantize_nvfp4 for the format and the tiled layout. */
+typedef enum { LMOE_EXPERTS_BF16 = 0, LMOE_EXPERTS_NVFP4 = 1 } lmoe_expert_format;
 
 typedef struct {
     int hidden;              /* H (multiple of 64)                               */
@@ -75,8 +80,10 @@ typedef struct {
     float routed_scaling_factor;
     lmoe_dtype x_dtype;      /* dtype of x                                       */
     lmoe_mode mode;          /* BF16 (tensor cores) or FP32 (validation)         */
+    lmoe_expert_format expert_format;  /* BF16 (default) or NVFP4               */
 } lmoe_config;
-/* Supported: E <= 1024, k <= min(64, Gk * E / G), E / G >= 2 when G > 1. */
+/* Supported: E <= 1024, k <= min(64, Gk * E / G), E / G >= 2 when G > 1.
+ * NVFP4 experts: mode LMOE_MODE_BF16, I and L multiples of 128. */
 
 typedef struct {
     const void* router_w;       /* [E, H]  bf16                                   */
@@ -87,6 +94,14 @@ typedef struct {
     const void* down_w;         /* [E, L, I] bf16 expert down_proj                */
     const void* shared_up_w;    /* [Is, H] bf16 shared expert up_proj             */
     const void* shared_down_w;  /* [H, Is] bf16 shared expert down_proj           */
+    /* NVFP4 experts only (expert_format = LMOE_EXPERTS_NVFP4; ignored otherwise):
+     * up_w and down_w then hold E2M1 codes, E*I*L/2 bytes each, in the tiled
+     * layout of latentmoe_quantize_nvfp4 (up: E matrices of [I, L]; down: E
+     * matrices of [L, I]), and these hold their scales.                        */
+    const void* up_sf;          /* E4M3 block scales of up_w, E*I*L/16 bytes      */
+    const void* down_sf;        /* E4M3 block scales of down_w, E*L*I/16 bytes    */
+    const float* up_gs;         /* [E] fp32 matrix scale of each expert's up_w    */
+    const float* down_gs;       /* [E] fp32 matrix scale of each expert's down_w  */
 } lmoe_weights;
 
 typedef struct lmoe_handle lmoe_handle;
@@ -124,6 +139,29 @@ lmoe_status latentmoe_forward_block(lmoe_handle* h, const void* x, int T, const 
                                     float* y, void* ws, size_t ws_bytes, void* stream, int32_t* topk_idx,
                                     float* topk_w, int32_t* expert_counts);
 
+/* NVFP4 quantisation of n_mat bf16 matrices [R, K] (w, row-major, contiguous;
+ * e.g. all E expert up_proj weights with R = I, K = L). Format: E2M1 elements
+ * (bit 3 sign, 2 exponent bits with bias 1, 1 mantissa bit: 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6), one E4M3 scale S per 16 consecutive elements along K (bias 7,
+ * 3 mantissa bits, subnormals, max 448), one fp32 scale g per matrix; the
+ * element's value is code * S * g. Recipe, every step an fp32 operation
+ * rounded to nearest even:
+ *   g = amax(matrix) / 2688 (1 if the matrix is zero)
+ *   S = nearest E4M3 to (amax(block) / g) / 6, saturating at 448
+ *   code = nearest E2M1 to w / (S * g), ties to the even mantissa, saturating
+ *          at 6, sign bit = (w / (S * g) < 0); a block with S = 0 gets code 0.
+ * Layout, in tiles of 128 rows x 64 K (gr = m * R + r is the global row):
+ *   tile = (gr / 128) * (K / 64) + k / 64
+ *   codes[tile * 4096 + (gr % 128) * 32 + (k % 64) / 2], element k even in
+ *   the low nibble;  sf[tile * 512 + (gr % 128) * 4 + (k % 64) / 16].
+ * codes (n_mat*R*K/2 bytes), sf (n_mat*R*K/16 bytes) and gs ([n_mat] fp32)
+ * are device memory written by the call; w, codes and sf 16-byte aligned.
+ * R % 128 == 0 and K % 64 == 0, else LMOE_ERR_UNSUPPORTED. Asynchronous on
+ * `stream`; deterministic. Needs no handle: a weight-conversion step run once
+ * before latentmoe_create. */
+lmoe_status latentmoe_quantize_nvfp4(const void* w, long long n_mat, int R, int K, void* codes, void* sf, float* gs,
+                                     void* stream);
+
 /* Releases the handle (host memory only). */
 void latentmoe_destroy(lmoe_handle* h);
 
@@ -147,7 +185,10 @@ lmoe_status latentmoe_update_bias(lmoe_handle* h, const int32_t* expert_counts, 
 typedef enum {
     LMOE_OPT_GEMM_PATH = 0,      /* 0 auto, 1 tcgen05 prefill tiles (128 x BN per SM), 2 tcgen05
                                     decode (swap-AB) tiles, 3 SIMT fp32 kernels (validation),
-                                    4 prefill tiles of 256 x 256 on 2-SM pairs (cta_group::2)     */
+                                    4 prefill tiles of 256 x 256 on 2-SM pairs (cta_group::2).
+                                    NVFP4 expert GEMMs always run weight-stationary tiles (32
+                                    tokens at decode sizes, else 128); the option then applies to
+                                    the dense GEMMs, and 3 is unsupported (LMOE_ERR_UNSUPPORTED). */
     LMOE_OPT_ROUTER_FP64_ALL = 1,/* 1: every token's logits recomputed in fp64 (validation)      */
     LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin for the fp64 re-check, in 1e-9 units        */
     LMOE_OPT_SPIN_LIMIT = 3      /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */

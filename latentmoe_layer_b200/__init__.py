@@ -21,24 +21,28 @@ LMOE_OK, LMOE_ERR_INVALID_ARG, LMOE_ERR_UNSUPPORTED, LMOE_ERR_WORKSPACE, LMOE_ER
     LMOE_ERR_INTERNAL = range(7)
 LMOE_BF16, LMOE_FP32 = 0, 1
 LMOE_MODE_BF16, LMOE_MODE_FP32 = 0, 1
+LMOE_EXPERTS_BF16, LMOE_EXPERTS_NVFP4 = 0, 1
 OPT_GEMM_PATH, OPT_ROUTER_FP64_ALL, OPT_FLAG_DELTA, OPT_SPIN_LIMIT = range(4)
 GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
-           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias", "latentmoe_forward_block"]
+           "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias", "latentmoe_forward_block",
+           "latentmoe_quantize_nvfp4"]
 
 
 class lmoe_config(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("latent", ctypes.c_int), ("num_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int),
                 ("expert_inter", ctypes.c_int), ("shared_inter", ctypes.c_int), ("max_tokens", ctypes.c_int),
-                ("routed_scaling_factor", ctypes.c_float), ("x_dtype", ctypes.c_int), ("mode", ctypes.c_int)]
+                ("routed_scaling_factor", ctypes.c_float), ("x_dtype", ctypes.c_int), ("mode", ctypes.c_int),
+                ("expert_format", ctypes.c_int)]
 
 
 class lmoe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
-                                                "shared_up_w", "shared_down_w")]
+                                                "shared_up_w", "shared_down_w", "up_sf", "down_sf", "up_gs",
+                                                "down_gs")]
 
 
 class lmoe_stats(ctypes.Structure):
@@ -81,10 +85,11 @@ def load():
     lib.latentmoe_route_noalloc.argtypes = [vp, vp, i32, vp, vp, vp, vp]
     lib.latentmoe_update_bias.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp]
     lib.latentmoe_forward_block.argtypes = [vp, vp, i32, vp, ctypes.c_float, vp, vp, sz, vp, vp, vp, vp]
+    lib.latentmoe_quantize_nvfp4.argtypes = [vp, ctypes.c_longlong, i32, i32, vp, vp, vp, vp]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
               "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias",
-              "latentmoe_forward_block"):
+              "latentmoe_forward_block", "latentmoe_quantize_nvfp4"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -150,6 +155,27 @@ def latentmoe_update_bias(h, counts, bias_in, eta, bias_out, maxvio, stream) -> 
     return load().latentmoe_update_bias(h, counts, bias_in, eta, bias_out, maxvio, stream)
 
 
+def latentmoe_quantize_nvfp4(w, n_mat, R, K, codes, sf, gs, stream) -> int:
+    return load().latentmoe_quantize_nvfp4(w, n_mat, R, K, codes, sf, gs, stream)
+
+
+def quantize_nvfp4(w):
+    """NVFP4 of a bf16 CUDA tensor [n_mat, R, K] on the current stream. Returns
+    (codes uint8 [n_mat*R*K/2], sf uint8 [n_mat*R*K/16], gs float32 [n_mat]) in
+    the library's tiled layout (include/latentmoe.h)."""
+    import torch
+    n_mat, R, K = w.shape
+    assert w.is_cuda and w.dtype == torch.bfloat16 and w.is_contiguous()
+    codes = torch.empty(n_mat * R * K // 2, dtype=torch.uint8, device=w.device)
+    sf = torch.empty(n_mat * R * K // 16, dtype=torch.uint8, device=w.device)
+    gs = torch.empty(n_mat, dtype=torch.float32, device=w.device)
+    s = latentmoe_quantize_nvfp4(_p(w), n_mat, R, K, _p(codes), _p(sf), _p(gs),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if s != LMOE_OK:
+        raise LmoeError(s, "latentmoe_quantize_nvfp4")
+    return codes, sf, gs
+
+
 def latentmoe_selftest_bounded_wait(h) -> int:
     return load().latentmoe_selftest_bounded_wait(h)
 
@@ -161,17 +187,21 @@ class LatentMoE:
     shape: an object with H, L, E, k, G, Gk, I, Is, s (e.g. synth.LayerShape).
     weights: dict of CUDA tensors router_w, e_bias, fc1_w, fc2_w, up_w, down_w,
     shared_up_w, shared_down_w (bf16, e_bias fp32). The tensors are borrowed.
+    expert_format LMOE_EXPERTS_NVFP4: up_w / down_w are the E2M1 code arrays of
+    quantize_nvfp4 and weights also holds up_sf, down_sf, up_gs, down_gs.
     """
 
-    def __init__(self, shape, weights: dict, max_tokens: int, x_f32: bool = False, mode: int = LMOE_MODE_BF16):
+    def __init__(self, shape, weights: dict, max_tokens: int, x_f32: bool = False, mode: int = LMOE_MODE_BF16,
+                 expert_format: int = LMOE_EXPERTS_BF16):
         import torch
         self.torch = torch
         self.shape = shape
         self.weights = weights
         cfg = lmoe_config(shape.H, shape.L, shape.E, shape.k, shape.G, shape.Gk, shape.I, shape.Is, max_tokens,
-                          float(shape.s), LMOE_FP32 if x_f32 else LMOE_BF16, mode)
-        w = lmoe_weights(*[_p(weights[n]) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
-                                                     "shared_up_w", "shared_down_w")])
+                          float(shape.s), LMOE_FP32 if x_f32 else LMOE_BF16, mode, expert_format)
+        w = lmoe_weights(*[_p(weights.get(n)) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
+                                                         "shared_up_w", "shared_down_w", "up_sf", "down_sf",
+                                                         "up_gs", "down_gs")])
         s, h = latentmoe_create(cfg, w)
         if s != LMOE_OK:
             raise LmoeError(s, "latentmoe_create")

@@ -40,8 +40,12 @@ def dense_weight_bytes(w) -> float:
     return 2.0 * (w.E * w.H + 2 * w.H * w.L + 2 * w.H * w.Is) + 4.0 * w.E
 
 
-def expert_bytes(w, distinct_experts: int) -> float:
-    """bf16 bytes of the expert weights a call must read: every hit expert's up and down once."""
+def expert_bytes(w, distinct_experts: int, nvfp4: bool = False) -> float:
+    """Bytes of the expert weights a call must read: every hit expert's up and down once.
+    bf16: 2 bytes per weight. NVFP4: half a byte per weight, one E4M3 scale byte per
+    16 weights and one fp32 matrix scale per matrix."""
+    if nvfp4:
+        return distinct_experts * 2 * (w.L * w.I * (0.5 + 1.0 / 16) + 4.0)
     return 2.0 * distinct_experts * 2 * w.L * w.I
 
 
@@ -50,6 +54,6 @@ def io_bytes(w, x_bytes_per_elem: int = 2) -> float:
     return w.T * w.H * (x_bytes_per_elem + 4.0)
 
 
-def min_bytes_per_call(w, distinct_experts: int) -> float:
+def min_bytes_per_call(w, distinct_experts: int, nvfp4: bool = False) -> float:
     """Compulsory HBM traffic of one call: weights touched once plus x and y."""
-    return dense_weight_bytes(w) + expert_bytes(w, distinct_experts) + io_bytes(w, 4 if w.x_f32 else 2)
+    return dense_weight_bytes(w) + expert_bytes(w, distinct_experts, nvfp4) + io_bytes(w, 4 if w.x_f32 else 2)

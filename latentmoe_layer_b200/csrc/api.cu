@@ -94,6 +94,10 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     p.pfx64 = take((E + 1) * 4);
     p.pfxdec = take((E + 1) * 4);
     p.pfx256 = take((E + 1) * 4);
+    p.rec32 = take((A / 32 + E) * 16);
+    p.rec64 = take((A / 64 + E) * 16);
+    p.rec128 = take((A / 128 + E) * 16);
+    p.rec256 = take((A / 256 + E) * 16);
     p.blockcounts = take((size_t)p.nblk * E * 4);
     p.perm = take(A * 4);
     p.slot = take(A * 4);
@@ -124,6 +128,10 @@ lmoe_status check_config(const lmoe_config* c) {
     if ((c->x_dtype != LMOE_BF16 && c->x_dtype != LMOE_FP32) ||
         (c->mode != LMOE_MODE_BF16 && c->mode != LMOE_MODE_FP32))
         return LMOE_ERR_INVALID_ARG;
+    if (c->expert_format != LMOE_EXPERTS_BF16 && c->expert_format != LMOE_EXPERTS_NVFP4) return LMOE_ERR_INVALID_ARG;
+    if (c->expert_format == LMOE_EXPERTS_NVFP4 &&
+        (c->mode != LMOE_MODE_BF16 || c->expert_inter % 128 || c->latent % 128))
+        return LMOE_ERR_UNSUPPORTED;  // weight tiles of 128 rows; tensor-core path only
     if (c->num_experts > kMaxE || c->n_group > kMaxG || c->top_k > kMaxK) return LMOE_ERR_UNSUPPORTED;
     if (c->n_group > 1 && c->num_experts / c->n_group < 2) return LMOE_ERR_UNSUPPORTED;
     if (c->hidden > 16384) return LMOE_ERR_UNSUPPORTED;  // fp64 router stages one x row in shared memory
@@ -131,12 +139,16 @@ lmoe_status check_config(const lmoe_config* c) {
     return LMOE_OK;
 }
 
-lmoe_status check_weights(const lmoe_weights* w) {
+lmoe_status check_weights(const lmoe_config& c, const lmoe_weights* w) {
     if (!w) return LMOE_ERR_INVALID_ARG;
     const void* ps[8] = {w->router_w, w->e_bias, w->fc1_w, w->fc2_w, w->up_w, w->down_w, w->shared_up_w,
                          w->shared_down_w};
     for (const void* p : ps)
         if (!p || !aligned(p, 16)) return LMOE_ERR_INVALID_ARG;
+    if (c.expert_format == LMOE_EXPERTS_NVFP4) {
+        if (!w->up_sf || !w->down_sf || !aligned(w->up_sf, 16) || !aligned(w->down_sf, 16)) return LMOE_ERR_INVALID_ARG;
+        if (!w->up_gs || !w->down_gs || !aligned(w->up_gs, 4) || !aligned(w->down_gs, 4)) return LMOE_ERR_INVALID_ARG;
+    }
     return LMOE_OK;
 }
 
@@ -207,6 +219,18 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
     if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
     if (pair) return launch_gemm_tc_pair(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
     return launch_gemm_tc(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
+}
+
+// Grouped expert GEMM with NVFP4 weights: only the activation operand goes
+// through a tensor map (box rows = the token tile); the weight tiles are
+// copied from the tiled code / scale arrays.
+cudaError_t run_gemm_nvfp4(Ctx& c, GemmProblem* pr, const Operand& act) {
+    const int bn = c.decode ? kDecodeTN : 128;
+    CUtensorMap map;
+    if (!encode_bf16(&map, act.ptr, act.rows, pr->kdim[0], bn)) return cudaErrorInvalidValue;
+    pr->a_map[0] = 0;
+    pr->b_map[0] = -1;
+    return launch_gemm_tc_nvfp4(&map, 1, pr, 1, bn, c.r, c.err, c.h->spin_limit, c.s);
 }
 
 GemmProblem make_problem(int grouped, int m_rows, int n, int epi, void* out, long long ldo) {
@@ -305,6 +329,10 @@ Ctx make_ctx(lmoe_handle* h, const Plan& p, void* ws, void* stream) {
     c.r.pfx64 = reinterpret_cast<const int*>(c.ws + p.pfx64);
     c.r.pfxdec = reinterpret_cast<const int*>(c.ws + p.pfxdec);
     c.r.pfx256 = reinterpret_cast<const int*>(c.ws + p.pfx256);
+    c.r.rec32 = reinterpret_cast<const int4*>(c.ws + p.rec32);
+    c.r.rec64 = reinterpret_cast<const int4*>(c.ws + p.rec64);
+    c.r.rec128 = reinterpret_cast<const int4*>(c.ws + p.rec128);
+    c.r.rec256 = reinterpret_cast<const int4*>(c.ws + p.rec256);
     c.r.E = h->cfg.num_experts;
     c.err = &reinterpret_cast<WsStats*>(c.ws + p.stats)->device_error;
     const lmoe_config& cf = h->cfg;
@@ -373,7 +401,8 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
     LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, ws_c + p.zperm, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
                                       reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
     mark(c, 3);
-    // 7: a = relu2(z_e W_up[e]^T)
+    const bool fp4 = cf.expert_format == LMOE_EXPERTS_NVFP4;
+    // 7: a = relu2(z_e W_up[e]^T)   (NVFP4: relu2(g_e * (z_e (codes * scales)^T)))
     {
         GemmProblem pr = make_problem(1, 0, I, epi_relu2, ws_c + p.aperm, I);
         pr.kdim[0] = L;
@@ -382,7 +411,14 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         pr.b_ptr[0] = h->w.up_w;
         Operand a[1][2] = {{{ws_c + p.zperm, A}, {nullptr, 0}}};
         Operand b[1][2] = {{{h->w.up_w, (long long)E * I}, {nullptr, 0}}};
-        LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
+        if (fp4) {
+            pr.wq_codes = static_cast<const uint8_t*>(h->w.up_w);
+            pr.wq_sf = static_cast<const uint8_t*>(h->w.up_sf);
+            pr.wscale = h->w.up_gs;
+            LMOE_LAUNCH(1, run_gemm_nvfp4(c, &pr, a[0][0]));
+        } else {
+            LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
+        }
     }
     mark(c, 4);
     // 8: o = w * (a_e W_down[e]^T)
@@ -395,7 +431,14 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         pr.b_ptr[0] = h->w.down_w;
         Operand a[1][2] = {{{ws_c + p.aperm, A}, {nullptr, 0}}};
         Operand b[1][2] = {{{h->w.down_w, (long long)E * L}, {nullptr, 0}}};
-        LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
+        if (fp4) {
+            pr.wq_codes = static_cast<const uint8_t*>(h->w.down_w);
+            pr.wq_sf = static_cast<const uint8_t*>(h->w.down_sf);
+            pr.wscale = h->w.down_gs;
+            LMOE_LAUNCH(1, run_gemm_nvfp4(c, &pr, a[0][0]));
+        } else {
+            LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
+        }
     }
     mark(c, 5);
     // 9: comb
@@ -469,7 +512,7 @@ lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe
     if (!out) return LMOE_ERR_INVALID_ARG;
     lmoe_status s = check_config(cfg);
     if (s != LMOE_OK) return s;
-    s = check_weights(w);
+    s = check_weights(*cfg, w);
     if (s != LMOE_OK) return s;
     if (!get_encoder()) return LMOE_ERR_CUDA;
     lmoe_handle* h = new (std::nothrow) lmoe_handle();
@@ -542,6 +585,7 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
     switch (opt) {
         case LMOE_OPT_GEMM_PATH:
             if (v < 0 || v > 4) return LMOE_ERR_INVALID_ARG;
+            if (v == 3 && h->cfg.expert_format == LMOE_EXPERTS_NVFP4) return LMOE_ERR_UNSUPPORTED;
             h->gemm_path = (int)v;
             return LMOE_OK;
         case LMOE_OPT_ROUTER_FP64_ALL:
@@ -578,6 +622,17 @@ lmoe_status latentmoe_update_bias(lmoe_handle* h, const int32_t* expert_counts, 
         return LMOE_ERR_INVALID_ARG;
     return cuda_status(launch_update_bias(expert_counts, bias_in, h->cfg.num_experts, (double)eta, bias_out, maxvio_out,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+lmoe_status latentmoe_quantize_nvfp4(const void* w, long long n_mat, int R, int K, void* codes, void* sf, float* gs,
+                                     void* stream) {
+    if (n_mat < 0 || R <= 0 || K <= 0) return LMOE_ERR_INVALID_ARG;
+    if (n_mat == 0) return LMOE_OK;
+    if (!w || !codes || !sf || !gs || !aligned(w, 16) || !aligned(codes, 16) || !aligned(sf, 16) || !aligned(gs, 4))
+        return LMOE_ERR_INVALID_ARG;
+    if (R % 128 || K % 64 || n_mat > 65535 || (long long)R * K > (1LL << 40) / n_mat) return LMOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quantize_nvfp4(static_cast<const uint16_t*>(w), n_mat, R, K, static_cast<uint8_t*>(codes),
+                                             static_cast<uint8_t*>(sf), gs, static_cast<cudaStream_t>(stream)));
 }
 
 lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n) {

@@ -73,10 +73,11 @@ struct TileInfo {
     int rows;    // valid activation rows in this tile
     int wrow0;   // first weight row (row of B)
     int col0;    // first output column
+    int e;       // expert of a grouped tile (-1 for dense problems)
     bool half;   // non-swapped tile with <= 64 valid rows: M = 64 MMAs (the expert's ragged tail)
 };
 
-template <int BN, bool kSwap>
+template <int BN, bool kSwap, bool kFp4 = false>
 struct Shape {
     static constexpr int XR = 128;            // rows of the MMA A operand tile
     static constexpr int YR = BN;             // rows of the MMA B operand tile
@@ -94,10 +95,37 @@ struct Shape {
                                         : kCols <= 256 ? 256 : 512;
     static constexpr int kEpiWarps = BN >= 128 ? 8 : 4;  // two warps per TMEM lane quarter for wide tiles
     static constexpr int kColsPerThread = BN / (kEpiWarps / 4);
-    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    // NVFP4 weights (swap tiles): the 128 x 64 weight tile arrives as 4096 bytes of
+    // E2M1 codes and 512 bytes of E4M3 scales, and dequantisation warps write the
+    // bf16 operand tile from them.
+    static constexpr int kRawBytes = kFp4 ? 4096 + 512 : 0;
+    static constexpr int kTxBytes = kFp4 ? kRawBytes + kYBytes : kStageBytes;  // bytes the producer's copies carry
+    // Dequantisation warps, in groups that take alternate k-blocks so that
+    // several stages convert at once: 8 groups of 1 warp for decode tiles,
+    // 2 groups of 2 warps where the registers allow fewer warps.
+    static constexpr int kDeqWarps = !kFp4 ? 0 : BN <= 64 ? 8 : 4;
+    static constexpr int kDeqGroups = !kFp4 ? 1 : BN <= 64 ? 8 : 2;
+    static constexpr int kDeqGroupWarps = kFp4 ? kDeqWarps / kDeqGroups : 1;
+    static constexpr int kDeqItems = kFp4 ? 256 / (32 * kDeqGroupWarps) : 0;  // (row, half-row) items per thread
+    static constexpr int kThreads = 64 + 32 * (kEpiWarps + kDeqWarps);
     // per epilogue warp: one 32-row x 128-byte output box, 128-byte swizzled, for bulk tensor stores
     static constexpr int kStageOutBytes = kSwap ? 0 : 4096;
+    static constexpr int kBarBytes = 512;
+    static constexpr int kLutBytes = kFp4 ? 256 * 4 : 0;
+    static_assert(!kFp4 || kSwap, "NVFP4 weights sit on the MMA M side");
 };
+
+// Per-expert tile prefix and tile records of a grouped problem for activation
+// tiles of R rows.
+template <int R>
+__device__ __forceinline__ const int* grouped_prefix(const DeviceRouting& r) {
+    static_assert(R == 32 || R == 64 || R == 128 || R == 256, "activation tile rows");
+    return R == kDecodeTN ? r.pfxdec : R == 64 ? r.pfx64 : R == 128 ? r.pfx128 : r.pfx256;
+}
+template <int R>
+__device__ __forceinline__ const int4* grouped_records(const DeviceRouting& r) {
+    return R == kDecodeTN ? r.rec32 : R == 64 ? r.rec64 : R == 128 ? r.rec128 : r.rec256;
+}
 
 __device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
 
@@ -105,7 +133,7 @@ template <int BN, bool kSwap>
 __device__ __forceinline__ int total_tiles(const TcParams& P) {
     using S = Shape<BN, kSwap>;
     if (P.prob[0].grouped) {
-        const int* pfx = kSwap ? P.r.pfxdec : P.r.pfx128;
+        const int* pfx = grouped_prefix<S::kActRows>(P.r);
         return pfx[P.r.E] * n_col_tiles(P.prob[0], S::kOutCols);
     }
     return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
@@ -114,7 +142,9 @@ __device__ __forceinline__ int total_tiles(const TcParams& P) {
 // Tile t -> coordinates. Dense problems are rasterised in groups of kGroupM
 // row tiles (column tiles outer within a group) so that concurrently running
 // CTAs share both operands in L2. Grouped problems walk experts in order,
-// column tiles inner, so an expert's weights are read while its rows are hot.
+// column tiles inner, so an expert's weights are read while its rows are hot;
+// their row tiles come from the permutation's tile records (one 16-byte load,
+// instead of a dependent search over the per-expert prefix at every tile).
 template <int BN, bool kSwap>
 __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
     using S = Shape<BN, kSwap>;
@@ -123,20 +153,14 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         const GemmProblem& pr = P.prob[0];
         const int nct = n_col_tiles(pr, S::kOutCols);
         const int mt = t / nct, ct = t % nct;
-        const int* pfx = kSwap ? P.r.pfxdec : P.r.pfx128;
-        int lo = 0, hi = P.r.E;
-        while (hi - lo > 1) {
-            int mid = (lo + hi) >> 1;
-            if (__ldg(&pfx[mid]) <= mt) lo = mid;
-            else hi = mid;
-        }
-        const int e = lo;
-        const int off = __ldg(&P.r.offsets[e]), end = __ldg(&P.r.offsets[e + 1]);
+        const int4 rc = __ldg(grouped_records<S::kActRows>(P.r) + mt);
+        const int e = rc.x;
         ti.p = 0;
-        ti.row0 = off + (mt - __ldg(&pfx[e])) * S::kActRows;
-        ti.rows = min(S::kActRows, end - ti.row0);
+        ti.row0 = rc.y;
+        ti.rows = rc.z;
         ti.col0 = ct * S::kOutCols;
         ti.wrow0 = e * pr.b_rows_per_expert + ti.col0;
+        ti.e = e;
         ti.half = !kSwap && ti.rows <= 64;
         return ti;
     }
@@ -163,6 +187,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
     ti.rows = min(S::kActRows, pr.m_rows - ti.row0);
     ti.col0 = ct * S::kOutCols;
     ti.wrow0 = ti.col0;
+    ti.e = -1;
     ti.half = !kSwap && ti.rows <= 64;
     return ti;
 }
@@ -179,6 +204,11 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
                                                float (&acc)[CW], const CUtensorMap* omap, uint8_t* stage) {
     const int epi = pr.epi;
     const int lane = threadIdx.x & 31;
+    if (pr.wscale) {  // NVFP4 experts: h = g_e * (sum of code * block scale * activation)
+        const float g = __ldg(&pr.wscale[ti.e]);
+#pragma unroll
+        for (int i = 0; i < CW; ++i) acc[i] *= g;
+    }
     if (epi == EPI_RELU2_BF16 || epi == EPI_RELU2_F32) {
 #pragma unroll
         for (int i = 0; i < CW; ++i) {
@@ -288,22 +318,60 @@ __device__ __forceinline__ int tile_kblocks(const GemmProblem& pr) {
     return n;
 }
 
-template <int BN, int STAGES, bool kSwap>
-__global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
-    using S = Shape<BN, kSwap>;
+// ---------------------------------------------------------------- NVFP4
+// E2M1 codes -> bf16. Eight codes (one 32-bit word, element i in nibble i) give
+// four bf16 pairs. The three magnitude bits index two byte tables held in
+// registers (high and low byte of the bf16 value of 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+// with byte permutes; the sign bits are moved to bit 7 of the high bytes; the
+// block scale (bf16, both halves) multiplies the pair. code * scale has at most
+// 6 significant bits and lies in [2^-10, 2688], so the product is exact.
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t c, uint32_t scale2) {
+    constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;  // high bytes of magnitudes 0..3, 4..7
+    constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;  // low bytes
+    const uint32_t mag = c & 0x77777777u;
+    const uint32_t d = c << 4;  // bit 7 of byte j = sign of element 2j; bit 7 of c's byte j = sign of 2j + 1
+    const uint32_t mhi = mag >> 16;
+    const uint32_t h0 = prmt(kHi0, kHi1, mag) | (prmt(d, c, 0x5140u) & 0x80808080u);
+    const uint32_t l0 = prmt(kLo0, kLo1, mag);
+    const uint32_t h1 = prmt(kHi0, kHi1, mhi) | (prmt(d, c, 0x7362u) & 0x80808080u);
+    const uint32_t l1 = prmt(kLo0, kLo1, mhi);
+    uint4 o;
+    o.x = mul_bf16x2(prmt(l0, h0, 0x5140u), scale2);
+    o.y = mul_bf16x2(prmt(l0, h0, 0x7362u), scale2);
+    o.z = mul_bf16x2(prmt(l1, h1, 0x5140u), scale2);
+    o.w = mul_bf16x2(prmt(l1, h1, 0x7362u), scale2);
+    return o;
+}
+
+// bf16 value of an E4M3 byte (bias 7, 3 mantissa bits, subnormals m * 2^-9),
+// duplicated in both halves. Exact: E4M3 values need 4 significant bits.
+__device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+    if (b & 0x80u) v = -v;
+    const uint32_t h = __float_as_uint(v) >> 16;
+    return h | (h << 16);
+}
+
+template <int BN, int STAGES, bool kSwap, bool kFp4 = false>
+__global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+    using S = Shape<BN, kSwap, kFp4>;
     constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
     uint8_t* sX = smem;                                  // STAGES x kXBytes
     uint8_t* sY = smem + STAGES * S::kXBytes;            // STAGES x kYBytes
-    uint8_t* sOut = sY + STAGES * S::kYBytes;            // kEpiWarps x kStageOutBytes
+    uint8_t* sRaw = sY + STAGES * S::kYBytes;            // STAGES x kRawBytes (NVFP4 codes + scales)
+    uint8_t* sOut = sRaw + STAGES * S::kRawBytes;        // kEpiWarps x kStageOutBytes
     uint64_t* full = reinterpret_cast<uint64_t*>(sOut + S::kEpiWarps * S::kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* cfull = empty + STAGES;   // chunk accumulator ready (MMA -> epilogue)
     uint64_t* cempty = cfull + NB;      // chunk accumulator drained (epilogue -> MMA)
     uint64_t* done = cempty + NB;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* deq = done + 1;           // NVFP4: bf16 weight tile written (dequantisation -> MMA)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(deq + STAGES);
+    uint32_t* scale_lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(full) + S::kBarBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -316,8 +384,13 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
             mbar_init(&cempty[b], S::kEpiWarps);
         }
         mbar_init(done, 1);
+        if (kFp4)
+            for (int s = 0; s < STAGES; ++s) mbar_init(&deq[s], S::kDeqGroupWarps);
         fence_mbar_init();
     }
+    if (kFp4 && warp >= 2 + S::kEpiWarps)
+        for (int b = threadIdx.x - 32 * (2 + S::kEpiWarps); b < 256; b += 32 * S::kDeqWarps)
+            scale_lut[b] = e4m3_to_bf16x2((uint32_t)b);
     if (warp == 0 && lane == 0)
         for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
     if (warp == 1) {
@@ -348,8 +421,15 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-                    if (!kSwap) {
+                    mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
+                    if (kFp4) {
+                        // weight tile (128 rows x 64 K) of NVFP4 codes and scales; tokens by TMA
+                        const long long tile = (long long)(ti.wrow0 >> 7) * kb_n + kb;
+                        uint8_t* raw = sRaw + stage * S::kRawBytes;
+                        bulk_load(raw, pr.wq_codes + tile * 4096, 4096, &full[stage]);
+                        bulk_load(raw + 4096, pr.wq_sf + tile * 512, 512, &full[stage]);
+                        tma_load_2d(sY + stage * S::kYBytes, amap, &full[stage], kb * kBK, ti.row0);
+                    } else if (!kSwap) {
                         tma_load_2d(sX + stage * S::kXBytes, amap, &full[stage], kb * kBK, ti.row0);
                         tma_load_2d(sY + stage * S::kYBytes, bmap, &full[stage], kb * kBK, ti.wrow0);
                     } else {
@@ -390,7 +470,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                 const uint32_t d = tmem_base + (uint32_t)(buf * BN);
                 const int kb1 = min(kb_total, kb0 + CK);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
+                    if (!mbar_wait_bounded(kFp4 ? &deq[stage] : &full[stage], phase, P.spin, err)) {
                         ok = false;
                         break;
                     }
@@ -420,6 +500,64 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
         // all MMAs issued by this thread have completed before TMEM is freed
         umma_commit(done);
         mbar_wait_bounded(done, 0, 1u << 26, err);
+    } else if (kFp4 && warp >= 2 + S::kEpiWarps) {
+        // ------------------------------------------------ NVFP4 dequantisation
+        // Each thread converts (row, half-row) items of the 128 x 64 weight tile:
+        // 32 codes (16 bytes) and their two block scales -> four 16-byte chunks
+        // of the 128-byte-swizzled bf16 operand row (chunk j at (j ^ (row & 7)) * 16).
+        // Group g takes the k-blocks c with c % kDeqGroups == g (c counts the
+        // CTA's k-blocks in the producer's order), so groups convert different
+        // stages at the same time.
+        const int dw = warp - (2 + S::kEpiWarps);
+        const int grp = dw / S::kDeqGroupWarps;
+        const int gt = (dw % S::kDeqGroupWarps) * 32 + lane;  // thread within the group
+        uint32_t c = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, kSwap>(P, t);
+            const int kb_total = tile_kblocks(P.prob[ti.p]);
+            for (int kb = 0; kb < kb_total; ++kb, ++c) {
+                if ((int)(c % S::kDeqGroups) != grp) continue;
+                const int stage = (int)(c % STAGES);
+                const uint32_t phase = (c / STAGES) & 1u;
+                if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* raw = sRaw + stage * S::kRawBytes;
+                uint8_t* dst = sX + stage * S::kXBytes;
+                constexpr int NI = S::kDeqItems > 0 ? S::kDeqItems : 1;  // (the branch is dead without NVFP4)
+#pragma unroll
+                for (int i0 = 0; i0 < NI; i0 += 2) {  // two items' loads first, so their conversions overlap
+                    constexpr int NJ = NI >= 2 ? 2 : 1;
+                    uint4 cw[NJ];
+                    uint32_t sA[NJ], sB[NJ];
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int it = gt + (i0 + j) * 32 * S::kDeqGroupWarps, r = it >> 1, hh = it & 1;
+                        cw[j] = *reinterpret_cast<const uint4*>(raw + r * 32 + hh * 16);
+                        const uint32_t sb = *reinterpret_cast<const uint16_t*>(raw + 4096 + r * 4 + hh * 2);
+                        sA[j] = scale_lut[sb & 0xFFu];
+                        sB[j] = scale_lut[sb >> 8];
+                    }
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int it = gt + (i0 + j) * 32 * S::kDeqGroupWarps, r = it >> 1, hh = it & 1;
+                        uint8_t* row = dst + r * 128;
+                        const int sw = r & 7, j0 = 4 * hh;
+                        const uint4 o0 = e2m1x8_to_bf16(cw[j].x, sA[j]), o1 = e2m1x8_to_bf16(cw[j].y, sA[j]);
+                        const uint4 o2 = e2m1x8_to_bf16(cw[j].z, sB[j]), o3 = e2m1x8_to_bf16(cw[j].w, sB[j]);
+                        st_shared_v4(row + (((j0 + 0) ^ sw) << 4), o0);
+                        st_shared_v4(row + (((j0 + 1) ^ sw) << 4), o1);
+                        st_shared_v4(row + (((j0 + 2) ^ sw) << 4), o2);
+                        st_shared_v4(row + (((j0 + 3) ^ sw) << 4), o3);
+                    }
+                }
+                fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&deq[stage]);
+            }
+        }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
         const int ew = warp - 2;
@@ -536,23 +674,17 @@ __device__ __forceinline__ int pair_total_tiles(const TcParams& P) {
 // for the second CTA of a short tile), B rows wrow0 .. wrow0+127, output
 // columns col0 .. col0+255.
 __device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32_t rank) {
-    int p = 0, prow0, prows, ct, wbase = 0;
+    int p = 0, prow0, prows, ct, wbase = 0, e = -1;
     if (P.prob[0].grouped) {
         const GemmProblem& pr = P.prob[0];
         const int nct = pr.n / PairShape::BN;
         const int mt = t / nct;
         ct = t % nct;
-        const int* pfx = P.r.pfx256;
-        int lo = 0, hi = P.r.E;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (__ldg(&pfx[mid]) <= mt) lo = mid;
-            else hi = mid;
-        }
-        const int off = __ldg(&P.r.offsets[lo]), end = __ldg(&P.r.offsets[lo + 1]);
-        prow0 = off + (mt - __ldg(&pfx[lo])) * 256;
-        prows = min(256, end - prow0);
-        wbase = lo * pr.b_rows_per_expert;
+        const int4 rc = __ldg(P.r.rec256 + mt);
+        prow0 = rc.y;
+        prows = rc.z;
+        wbase = rc.x * pr.b_rows_per_expert;
+        e = rc.x;
     } else {
         if (P.nprob > 1 && t >= P.dense_tiles[0]) {
             t -= P.dense_tiles[0];
@@ -574,6 +706,7 @@ __device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32
     ti.rows = min(128, prows - (int)rank * 128);
     ti.col0 = ct * PairShape::BN;
     ti.wrow0 = wbase + ti.col0 + (int)rank * 128;
+    ti.e = e;
     ti.half = false;
     return ti;
 }
@@ -759,21 +892,23 @@ __global__ void __launch_bounds__(PairShape::kThreads, 1) k_gemm_tc_pair(const _
     if (warp == 1) tmem_dealloc_pair(tmem_base, S::kTmemCols);
 }
 
-template <int BN, int STAGES, bool kSwap>
+template <int BN, int STAGES, bool kSwap, bool kFp4>
 constexpr size_t smem_bytes() {
-    using S = Shape<BN, kSwap>;
-    return 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 256;
+    using S = Shape<BN, kSwap, kFp4>;
+    return 1024 + (size_t)STAGES * (S::kStageBytes + S::kRawBytes) + (size_t)S::kEpiWarps * S::kStageOutBytes +
+           S::kBarBytes + S::kLutBytes;
 }
 
-template <int BN, int STAGES, bool kSwap>
+template <int BN, int STAGES, bool kSwap, bool kFp4 = false>
 cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
-    constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
+    using S = Shape<BN, kSwap, kFp4>;
+    constexpr size_t smem = smem_bytes<BN, STAGES, kSwap, kFp4>();
     static_assert(smem <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * Shape<BN, kSwap>::kBufs + 1) * 8 + 4 <= 256, "barrier area");
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    static_assert((3 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= S::kBarBytes, "barrier area");
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap, kFp4>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_gemm_tc<BN, STAGES, kSwap><<<grid, Shape<BN, kSwap>::kThreads, smem, s>>>(P);
+    k_gemm_tc<BN, STAGES, kSwap, kFp4><<<grid, S::kThreads, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -888,6 +1023,22 @@ cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const Gemm
         if (grid < 1) return cudaSuccess;
     }
     return launch_impl<kDecodeTN, 10, true>(P, grid, s);
+}
+
+// Grouped expert GEMMs with NVFP4 weights: weight-stationary tiles (128 weight
+// rows on the MMA M side), bn = 32 tokens per tile (decode) or 128 (prefill).
+cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
+                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    if (nprob != 1 || !probs[0].grouped || probs[0].nseg != 1 || !probs[0].wq_codes || !probs[0].wq_sf)
+        return cudaErrorInvalidValue;
+    TcParams P;
+    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
+    const int grid = tc_num_sms();
+    switch (bn) {
+        case kDecodeTN: return launch_impl<kDecodeTN, 8, true, true>(P, grid, s);
+        case 128: return launch_impl<128, 6, true, true>(P, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // ---------------------------------------------------------------- self-test

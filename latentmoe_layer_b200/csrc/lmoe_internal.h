@@ -55,6 +55,12 @@ struct GemmProblem {
     const float* row_scale; // EPI_SCALE_F32
     int out_map;            // tensor map of `out` for bulk tensor stores (-1: plain stores)
     const uint16_t* resid;  // EPI_F32 only: bf16 [rows, ldo] added to the result (block residual)
+    // NVFP4 weights (grouped swap-AB problems only): B is given as E2M1 codes and
+    // E4M3 block scales in 128-row x 64-K tiles, and each expert's accumulator is
+    // multiplied by wscale[e] before the epilogue operation.
+    const uint8_t* wq_codes;  // tile t at wq_codes + 4096 t
+    const uint8_t* wq_sf;     // tile t at wq_sf + 512 t
+    const float* wscale;      // [E] matrix scale per expert
 };
 
 struct DeviceRouting {
@@ -63,14 +69,21 @@ struct DeviceRouting {
     const int* pfx64;       // [E+1] prefix of ceil(count/64)
     const int* pfxdec;      // [E+1] prefix of ceil(count/kDecodeTN)
     const int* pfx256;      // [E+1] prefix of ceil(count/256) (2-SM pair tiles)
+    // Tile records per activation-tile height R = 32, 64, 128, 256: entry j of
+    // recR is {expert, first permuted row, rows, 0} of the j-th R-row tile in
+    // expert order (pfxR[E] entries), so a GEMM finds its tile with one load.
+    const int4* rec32;
+    const int4* rec64;
+    const int4* rec128;
+    const int4* rec256;
     int E;
 };
 
 // Workspace carving for one call.
 struct Plan {
     size_t total;
-    size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, blockcounts, perm,
-        slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as;
+    size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64,
+        rec128, rec256, blockcounts, perm, slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as;
     int T, A, nblk;
 };
 
@@ -103,6 +116,10 @@ cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmPr
                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
 cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
                                   const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
+cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
+                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
+cudaError_t launch_quantize_nvfp4(const uint16_t* w, long long n_mat, int R, int K, uint8_t* codes, uint8_t* sf,
+                                  float* gs, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* err, unsigned spin_limit, cudaStream_t s);
 int tc_num_sms();
 }  // namespace lmoe

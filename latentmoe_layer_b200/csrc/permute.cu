@@ -79,7 +79,8 @@ __device__ void block_scan4(int4& v, int4* warp_tot) {
 __global__ void __launch_bounds__(1024)
     k_scan(int* __restrict__ blockcounts, int nblk, int E, int* __restrict__ counts, int32_t* __restrict__ counts_out,
            int* __restrict__ offsets, int* __restrict__ pfx128, int* __restrict__ pfx64, int* __restrict__ pfxdec,
-           int* __restrict__ pfx256, WsStats* __restrict__ st) {
+           int* __restrict__ pfx256, int4* __restrict__ rec32, int4* __restrict__ rec64, int4* __restrict__ rec128,
+           int4* __restrict__ rec256, WsStats* __restrict__ st) {
     __shared__ int4 warp_tot[32];
     __shared__ int red[2];
     const int e = threadIdx.x;
@@ -126,6 +127,17 @@ __global__ void __launch_bounds__(1024)
             pfx64[E] = incl.z;
             pfxdec[E] = incl.w;
         }
+    }
+    // tile records: the j-th R-row tile of expert e starts at row offset + j R
+    if (e < E) {
+        const int off = incl.x - v.x;
+        int4* recs[4] = {rec32 + (incl.w - v.w), rec64 + (incl.z - v.z), rec128 + (incl.y - v.y),
+                         rec256 + (incl2.x - v2.x)};
+        const int rows[4] = {kDecodeTN, 64, 128, 256};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            for (int j = 0; j * rows[q] < run; ++j)
+                recs[q][j] = make_int4(e, off + j * rows[q], min(rows[q], run - j * rows[q]), 0);
     }
     __syncthreads();
     if (e == 0) {
@@ -342,7 +354,9 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
     k_scan<<<1, 1024, 0, s>>>(bc, p.nblk, E, reinterpret_cast<int*>(ws + p.counts), counts_out,
                               reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
                               reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
-                              reinterpret_cast<int*>(ws + p.pfx256), reinterpret_cast<WsStats*>(ws + p.stats));
+                              reinterpret_cast<int*>(ws + p.pfx256), reinterpret_cast<int4*>(ws + p.rec32),
+                              reinterpret_cast<int4*>(ws + p.rec64), reinterpret_cast<int4*>(ws + p.rec128),
+                              reinterpret_cast<int4*>(ws + p.rec256), reinterpret_cast<WsStats*>(ws + p.stats));
     const size_t scatter_smem = (size_t)(kScatterWarps * E + kChunk * k) * sizeof(int);
     if (scatter_smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);

@@ -57,8 +57,12 @@ ULTRA_SKEW = LayerShape("ultra_skew", T=8192, H=8192, L=2048, E=512, k=22, G=8, 
 # the same ~704 rows per expert, but 64 experts (~3 GB of weights) so that a
 # multi-pass ncu capture stays small.
 PROBE_E64 = LayerShape("probe_e64", T=2048, H=8192, L=2048, E=64, k=22, G=8, Gk=4, I=5120, Is=10240)
+# Decode-sized counterpart (64 tokens, ~22 per expert as in ultra_decode's swap-AB
+# tiles), 2.7 GB of bf16 expert weights: small enough for a full profiler capture.
+PROBE_DECODE_E64 = LayerShape("probe_decode_e64", T=64, H=8192, L=2048, E=64, k=22, G=8, Gk=4, I=5120, Is=10240)
 
-WORKLOADS = {w.name: w for w in (TINY, NANO_DECODE, ULTRA_DECODE, ULTRA_PREFILL, ULTRA_SKEW, PROBE_E64)}
+WORKLOADS = {w.name: w for w in (TINY, NANO_DECODE, ULTRA_DECODE, ULTRA_PREFILL, ULTRA_SKEW, PROBE_E64,
+                                 PROBE_DECODE_E64)}
 
 # Stream ids of the generator, one per tensor.
 TID_X, TID_ROUTER, TID_BIAS, TID_FC1, TID_FC2, TID_UP, TID_DOWN, TID_SUP, TID_SDOWN = range(1, 10)

@@ -48,8 +48,9 @@ def good_cfg(**kw):
     return lm.lmoe_config(**c)
 
 
-def fake_weights(addr=0x10000):
-    return lm.lmoe_weights(*([addr] * 8))
+def fake_weights(addr=0x10000, nvfp4_addr=None):
+    extra = addr if nvfp4_addr is None else nvfp4_addr
+    return lm.lmoe_weights(*([addr] * 8 + [extra] * 4))
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -71,6 +72,35 @@ def fake_weights(addr=0x10000):
 def test_invalid_configs_rejected_before_any_cuda_call(lib, kw, status):
     s, h = lm.latentmoe_create(good_cfg(**kw), fake_weights())
     assert s == status and not h.value
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(expert_format=7), lm.LMOE_ERR_INVALID_ARG),
+    (dict(expert_format=lm.LMOE_EXPERTS_NVFP4, latent=128, mode=lm.LMOE_MODE_FP32), lm.LMOE_ERR_UNSUPPORTED),
+    (dict(expert_format=lm.LMOE_EXPERTS_NVFP4), lm.LMOE_ERR_UNSUPPORTED),                # L = 64: not 128 rows
+    (dict(expert_format=lm.LMOE_EXPERTS_NVFP4, latent=128, expert_inter=192), lm.LMOE_ERR_UNSUPPORTED),
+])
+def test_nvfp4_configs_rejected_before_any_cuda_call(lib, kw, status):
+    s, h = lm.latentmoe_create(good_cfg(**kw), fake_weights())
+    assert s == status and not h.value
+
+
+def test_nvfp4_weights_need_scales(lib):
+    cfg = good_cfg(expert_format=lm.LMOE_EXPERTS_NVFP4, latent=128)
+    for bad in (0, 0x10008):
+        s, h = lm.latentmoe_create(cfg, fake_weights(nvfp4_addr=bad))
+        assert s == lm.LMOE_ERR_INVALID_ARG and not h.value
+
+
+def test_quantize_nvfp4_argument_checks(lib):
+    q, st = lm.latentmoe_quantize_nvfp4, None
+    assert q(0x10000, 0, 128, 64, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_OK          # nothing to do
+    assert q(None, 1, 128, 64, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_ERR_INVALID_ARG
+    assert q(0x10008, 1, 128, 64, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_ERR_INVALID_ARG
+    assert q(0x10000, 1, 128, 64, 0x10000, 0x10000, 0x10002, st) == lm.LMOE_ERR_INVALID_ARG
+    assert q(0x10000, -1, 128, 64, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_ERR_INVALID_ARG
+    assert q(0x10000, 1, 64, 64, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_ERR_UNSUPPORTED
+    assert q(0x10000, 1, 128, 96, 0x10000, 0x10000, 0x10000, st) == lm.LMOE_ERR_UNSUPPORTED
 
 
 def test_null_or_misaligned_weights_rejected(lib):
