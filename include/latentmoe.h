@@ -201,6 +201,8 @@ typedef struct {
     int max_expert_tokens;  /* largest per-expert token count                   */
     int device_error;       /* lmoe_status recorded by a device-side check      */
     int kernel_launches;    /* kernels the last route/forward call on the handle launched */
+    int cuda_error;         /* cudaError_t of the last CUDA runtime call on the handle that
+                               failed (a call that returned LMOE_ERR_CUDA), 0 if none     */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */
@@ -233,7 +235,9 @@ lmoe_status latentmoe_route_noalloc(lmoe_handle* h, const void* x, int T, int32_
  * stage boundary i: 0 start, 1 routing done (router GEMM, selection, fp64
  * re-check, permutation), 2 input GEMM (fc1 + shared up) done, 3 gather done,
  * 4 expert up GEMM done, 5 expert down GEMM done, 6 combine done, 7 output
- * GEMM done. NULL turns it off. The events are borrowed. */
+ * GEMM done. NULL turns it off. The events are borrowed and must exist (a
+ * NULL event among the first 8 returns LMOE_ERR_INVALID_ARG); a record that
+ * fails is skipped and does not fail the call it times. */
 lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n);
 
 /* Runs one kernel that waits, with the handle's spin limit, on an mbarrier

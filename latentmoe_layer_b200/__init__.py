@@ -48,7 +48,7 @@ class lmoe_weights(ctypes.Structure):
 class lmoe_stats(ctypes.Structure):
     _fields_ = [("flagged_tokens", ctypes.c_int), ("distinct_experts", ctypes.c_int),
                 ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int),
-                ("kernel_launches", ctypes.c_int)]
+                ("kernel_launches", ctypes.c_int), ("cuda_error", ctypes.c_int)]
 
 
 class LmoeError(RuntimeError):

@@ -252,7 +252,10 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 #define LMOE_TRY(expr)                                   \
     do {                                                 \
         cudaError_t _e = (expr);                         \
-        if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
+        if (_e != cudaSuccess) {                         \
+            c.h->last_cuda_error = (int)_e;              \
+            return LMOE_ERR_CUDA;                        \
+        }                                                \
     } while (0)
 
 // Launch `expr`, which starts `n` kernels, and count them.
@@ -262,9 +265,13 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
         c.h->launches += (n);         \
     } while (0)
 
+// Stage marker (latentmoe_set_profile_events). A failed record must not leave
+// a pending runtime error for the next launch check to report, so it is
+// consumed here: a marker never fails the call it times.
 void mark(const Ctx& c, int i) {
-    if (c.h->prof_events && i < c.h->prof_n)
-        cudaEventRecord(static_cast<cudaEvent_t>(c.h->prof_events[i]), c.s);
+    if (c.h->prof_events && i < c.h->prof_n &&
+        cudaEventRecord(static_cast<cudaEvent_t>(c.h->prof_events[i]), c.s) != cudaSuccess)
+        (void)cudaGetLastError();
 }
 
 __attribute__((unused)) lmoe_status take_device_error(lmoe_handle* h) {
@@ -612,6 +619,7 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
     out->max_expert_tokens = st.max_count;
     out->device_error = st.device_error;
     out->kernel_launches = h->launches;
+    out->cuda_error = h->last_cuda_error;
     return LMOE_OK;
 }
 
@@ -637,6 +645,8 @@ lmoe_status latentmoe_quantize_nvfp4(const void* w, long long n_mat, int R, int 
 
 lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n) {
     if (!h || (events && n < 8)) return LMOE_ERR_INVALID_ARG;
+    for (int i = 0; events && i < 8; ++i)
+        if (!events[i]) return LMOE_ERR_INVALID_ARG;  // e.g. a framework event not created yet
     h->prof_events = events;
     h->prof_n = events ? n : 0;
     return LMOE_OK;

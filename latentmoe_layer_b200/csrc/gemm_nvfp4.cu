@@ -1,0 +1,347 @@
+// gemm_nvfp4.cu -- grouped expert GEMMs whose weights are NVFP4.
+//
+// The routed experts' up and down projections are the NVFP4 layers of the
+// pages' model ("Nemotron 3 Ultra 架构 QA", Q1.3 and Q8.1). Weights are E2M1
+// codes with one E4M3 scale per 16 along K and one fp32 scale per matrix
+// (layout in latentmoe.h), activations stay bf16: each 128 x 64 weight tile is
+// expanded exactly into bf16 in shared memory and multiplied on the tensor
+// cores (tcgen05.mma kind::f16, fp32 accumulation in TMEM), so the arithmetic
+// is that of the bf16 path applied to the dequantised weights.
+//
+// Weight-stationary tiles: MMA M = 128 weight rows, N = BN tokens of one
+// expert (BN = 32 at decode sizes, 128 otherwise). One ring of stages, each
+// holding KB k-blocks of 64: the token tiles (TMA, 128-byte swizzle), the
+// codes and scales (bulk copies), and the bf16 weight tiles the
+// dequantisation warps write from them. Every barrier wait and commit sits on
+// the path of a 32-token tile, whose tensor-core work per k-block is short,
+// so a stage carries several k-blocks to spread that cost.
+// Roles: warp 0 producer, warp 1 MMA issuer and TMEM owner, then the epilogue
+// warps (TMEM chunk drains, as in the bf16 kernel), then dequantisation warps
+// in G groups that take the stages in turn.
+#include "gemm_common.cuh"
+
+namespace lmoe {
+namespace {
+
+// E2M1 codes -> bf16. Eight codes (one 32-bit word, element i in nibble i) give
+// four bf16 pairs. The three magnitude bits index two byte tables held in
+// registers (high and low byte of the bf16 value of 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+// with byte permutes; the sign bits are moved to bit 7 of the high bytes; the
+// block scale (bf16, both halves) multiplies the pair. code * scale has at most
+// 6 significant bits and lies in [2^-10, 2688], so the product is exact.
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t c, uint32_t scale2) {
+    constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;  // high bytes of magnitudes 0..3, 4..7
+    constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;  // low bytes
+    const uint32_t mag = c & 0x77777777u;
+    const uint32_t d = c << 4;  // bit 7 of byte j = sign of element 2j; bit 7 of c's byte j = sign of 2j + 1
+    const uint32_t mhi = mag >> 16;
+    const uint32_t h0 = prmt(kHi0, kHi1, mag) | (prmt(d, c, 0x5140u) & 0x80808080u);
+    const uint32_t l0 = prmt(kLo0, kLo1, mag);
+    const uint32_t h1 = prmt(kHi0, kHi1, mhi) | (prmt(d, c, 0x7362u) & 0x80808080u);
+    const uint32_t l1 = prmt(kLo0, kLo1, mhi);
+    uint4 o;
+    o.x = mul_bf16x2(prmt(l0, h0, 0x5140u), scale2);
+    o.y = mul_bf16x2(prmt(l0, h0, 0x7362u), scale2);
+    o.z = mul_bf16x2(prmt(l1, h1, 0x5140u), scale2);
+    o.w = mul_bf16x2(prmt(l1, h1, 0x7362u), scale2);
+    return o;
+}
+
+// bf16 value of an E4M3 byte (bias 7, 3 mantissa bits, subnormals m * 2^-9),
+// duplicated in both halves. Exact: E4M3 values need 4 significant bits.
+__device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+    if (b & 0x80u) v = -v;
+    const uint32_t h = __float_as_uint(v) >> 16;
+    return h | (h << 16);
+}
+
+template <int BN, int STAGES, int KB, int G>
+struct Fp4Shape {
+    using T = Shape<BN, true>;                         // TMEM ring, epilogue split, token tile rows
+    static constexpr int kTokBytes = BN * kBK * 2;     // token tile of one k-block, BN rows x 128 bytes
+    static constexpr int kOpBytes = 128 * kBK * 2;     // bf16 weight tile of one k-block
+    // stage: KB token tiles | KB bf16 weight tiles | KB x 4096 code bytes | KB x 512 scale bytes
+    static constexpr int kOffOp = KB * kTokBytes;
+    static constexpr int kOffCodes = kOffOp + KB * kOpBytes;
+    static constexpr int kOffSf = kOffCodes + KB * 4096;
+    static constexpr int kStageBytes = (kOffSf + KB * 512 + 1023) & ~1023;  // swizzled tiles stay 1024-aligned
+    static constexpr int kTxBytes = KB * (kTokBytes + 4096 + 512);          // bytes the producer's copies carry
+    static constexpr int kDeqWarps = BN <= 64 ? 8 : 4;
+    static constexpr int kGroupWarps = kDeqWarps / G;
+    static constexpr int kItems = KB * 256 / (32 * kGroupWarps);  // (row, half-row) items per thread and stage
+    static constexpr int kThreads = 64 + 32 * (T::kEpiWarps + kDeqWarps);
+    static constexpr int kBarBytes = 1024;
+    static constexpr int kBars = 3 * STAGES + 2 * T::kBufs + 1;
+    static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStageBytes + kBarBytes + 1024;
+    static_assert(kBars * 8 + 4 <= kBarBytes, "barrier area");
+    static_assert(kDeqWarps % G == 0 && G <= STAGES && kItems % 2 == 0, "dequantisation groups");
+    static_assert(T::kChunkKB % KB == 0, "a chunk is whole stages");
+    static_assert(kSmem <= 232448, "shared memory");
+    static_assert(STAGES <= 32, "issued-load mask");
+};
+
+template <int BN, int STAGES, int KB, int G>
+__global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
+    k_gemm_nvfp4(const __grid_constant__ TcParams P) {
+    using F = Fp4Shape<BN, STAGES, KB, G>;
+    using S = typename F::T;
+    constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base_u32 = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * F::kStageBytes);  // copies landed (producer)
+    uint64_t* deq = full + STAGES;         // bf16 weight tiles written (dequantisation -> MMA)
+    uint64_t* empty = deq + STAGES;        // MMA done with the stage (MMA -> producer)
+    uint64_t* cfull = empty + STAGES;      // chunk accumulator ready (MMA -> epilogue)
+    uint64_t* cempty = cfull + NB;         // chunk accumulator drained (epilogue -> MMA)
+    uint64_t* done = cempty + NB;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint32_t* scale_lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(full) + F::kBarBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&deq[s], F::kGroupWarps);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&cfull[b], 1);
+            mbar_init(&cempty[b], S::kEpiWarps);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    const int dq0 = 2 + S::kEpiWarps;  // first dequantisation warp
+    if (warp >= dq0)
+        for (int b = threadIdx.x - 32 * dq0; b < 256; b += 32 * F::kDeqWarps) scale_lut[b] = e4m3_to_bf16x2((uint32_t)b);
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, S::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntiles = total_tiles<BN, true>(P);
+    const int kb_n = P.prob[0].kdim[0] / kBK;   // a multiple of KB (K is a multiple of 128)
+    const unsigned spin = P.spin;
+    int* err = P.err;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ producer
+        const CUtensorMap* amap = &P.maps[P.prob[0].a_map[0]];
+        const uint8_t* codes_g = P.prob[0].wq_codes;
+        const uint8_t* sf_g = P.prob[0].wq_sf;
+        uint32_t c = 0, issued = 0, issued_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, true>(P, t);
+            const long long tile0 = (long long)(ti.wrow0 >> 7) * kb_n;
+            for (int kb = 0; kb < kb_n; kb += KB, ++c) {
+                const int s = (int)(c % STAGES);
+                const uint32_t ph = (c / STAGES) & 1u;
+                if (!mbar_wait_bounded(&empty[s], ph ^ 1u, spin, err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + s * F::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], F::kTxBytes);
+#pragma unroll
+                for (int j = 0; j < KB; ++j) tma_load_2d(st + j * F::kTokBytes, amap, &full[s], (kb + j) * kBK, ti.row0);
+                bulk_load(st + F::kOffCodes, codes_g + (tile0 + kb) * 4096, KB * 4096, &full[s]);
+                bulk_load(st + F::kOffSf, sf_g + (tile0 + kb) * 512, KB * 512, &full[s]);
+                issued |= 1u << s;
+                issued_par = (issued_par & ~(1u << s)) | (ph << s);
+            }
+        }
+        // every copy this thread issued has landed before the CTA can exit
+        for (int s = 0; s < STAGES; ++s)
+            if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+        uint32_t c = 0, bphase = 0;
+        int buf = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int kb0 = 0; kb0 < kb_n && ok; kb0 += CK) {
+                if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+                const int kb1 = min(kb_n, kb0 + CK);
+                for (int kb = kb0; kb < kb1; kb += KB, ++c) {
+                    const int s = (int)(c % STAGES);
+                    if (!mbar_wait_bounded(&deq[s], (c / STAGES) & 1u, spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t* st = smem + s * F::kStageBytes;
+#pragma unroll
+                    for (int j = 0; j < KB; ++j) {
+                        const uint64_t adesc = sdesc_sw128(smem_u32(st + F::kOffOp + j * F::kOpBytes));
+                        const uint64_t bdesc = sdesc_sw128(smem_u32(st + j * F::kTokBytes));
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                                      (kb + j > kb0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&cfull[buf]);
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+        }
+        umma_commit(done);
+        mbar_wait_bounded(done, 0, 1u << 26, err);
+    } else if (warp >= dq0) {
+        // ------------------------------------------------ dequantisation
+        // Group g converts the stages c with c % G == g (c counts the CTA's
+        // stages in the producer's order). A thread converts (row, half-row)
+        // items: 32 codes (16 bytes) and their two block scales -> four 16-byte
+        // chunks of the 128-byte-swizzled bf16 row (chunk j at (j ^ (row & 7)) * 16).
+        // Item it of a stage: k-block it / 256 of the stage, row (it % 256) / 2.
+        const int dw = warp - dq0;
+        const int grp = dw / F::kGroupWarps;
+        const int gt = (dw % F::kGroupWarps) * 32 + lane;
+        uint32_t c = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int kb = 0; kb < kb_n; kb += KB, ++c) {
+                if ((int)(c % G) != grp) continue;
+                const int s = (int)(c % STAGES);
+                if (!mbar_wait_bounded(&full[s], (c / STAGES) & 1u, spin, err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + s * F::kStageBytes;
+#pragma unroll
+                for (int i0 = 0; i0 < F::kItems; i0 += 2) {  // two items' loads first, so their conversions overlap
+                    uint4 cw[2];
+                    uint32_t sA[2], sB[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int it = gt + (i0 + j) * 32 * F::kGroupWarps, kq = it >> 8, row = (it & 255) >> 1,
+                                  hh = it & 1;
+                        const uint8_t* codes = st + F::kOffCodes + kq * 4096;
+                        cw[j] = ld_shared_v4(codes + row * 32 + hh * 16);
+                        const uint32_t sb = ld_shared_u16(st + F::kOffSf + kq * 512 + row * 4 + hh * 2);
+                        sA[j] = ld_shared_u32(scale_lut + (sb & 0xFFu));
+                        sB[j] = ld_shared_u32(scale_lut + (sb >> 8));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int it = gt + (i0 + j) * 32 * F::kGroupWarps, kq = it >> 8, row = (it & 255) >> 1,
+                                  hh = it & 1;
+                        uint8_t* drow = st + F::kOffOp + kq * F::kOpBytes + row * 128;
+                        const int sw = row & 7, j0 = 4 * hh;
+                        const uint4 o0 = e2m1x8_to_bf16(cw[j].x, sA[j]), o1 = e2m1x8_to_bf16(cw[j].y, sA[j]);
+                        const uint4 o2 = e2m1x8_to_bf16(cw[j].z, sB[j]), o3 = e2m1x8_to_bf16(cw[j].w, sB[j]);
+                        st_shared_v4(drow + (((j0 + 0) ^ sw) << 4), o0);
+                        st_shared_v4(drow + (((j0 + 1) ^ sw) << 4), o1);
+                        st_shared_v4(drow + (((j0 + 2) ^ sw) << 4), o2);
+                        st_shared_v4(drow + (((j0 + 3) ^ sw) << 4), o3);
+                    }
+                }
+                fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&deq[s]);
+            }
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (as the bf16 swap tiles)
+        const GemmProblem& pr = P.prob[0];
+        const int ew = warp - 2;
+        const int q = warp & 3;                // TMEM lane quarter this warp may access
+        const int c0 = (ew >> 2) * CW;         // accumulator columns (tokens) this warp owns
+        const int lane_row = q * 32 + lane;
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN, true>(P, t);
+            float acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = 0.f;
+            for (int kb0 = 0; kb0 < kb_n; kb0 += CK) {
+                if (!mbar_wait_bounded(&cfull[buf], bphase, spin, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0);
+#pragma unroll
+                for (int cc = 0; cc < CW; cc += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(taddr + (uint32_t)cc, r0);
+                    if (cc + 16 < CW) tmem_ld16(taddr + (uint32_t)(cc + 16), r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[cc + i] += __uint_as_float(r0[i]);
+                    if (cc + 16 < CW) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[cc + 16 + i] += __uint_as_float(r1[i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cempty[buf]);
+                if (++buf == NB) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            epilogue_store<BN, true, CW>(pr, ti, lane_row, c0, acc, nullptr, nullptr);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+}
+
+template <int BN, int STAGES, int KB, int G>
+cudaError_t launch_nvfp4(const TcParams& P, int grid, cudaStream_t s) {
+    using F = Fp4Shape<BN, STAGES, KB, G>;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4<BN, STAGES, KB, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)F::kSmem);
+    if (e != cudaSuccess) return e;
+    k_gemm_nvfp4<BN, STAGES, KB, G><<<grid, F::kThreads, F::kSmem, s>>>(P);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Grouped expert GEMMs with NVFP4 weights, bn = 32 tokens per tile (decode) or 128.
+cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
+                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    if (nprob != 1 || !probs[0].grouped || probs[0].nseg != 1 || !probs[0].wq_codes || !probs[0].wq_sf)
+        return cudaErrorInvalidValue;
+    TcParams P;
+    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
+    const int grid = tc_num_sms();
+    switch (bn) {
+#ifndef LMOE_FP4_DEC
+#define LMOE_FP4_DEC 4, 2, 4   // stages, k-blocks per stage, dequantisation groups
+#endif
+        case kDecodeTN: return launch_nvfp4<kDecodeTN, LMOE_FP4_DEC>(P, grid, s);
+        case 128: return launch_nvfp4<128, 3, 2, 2>(P, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace lmoe

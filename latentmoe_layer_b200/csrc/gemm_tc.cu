@@ -34,344 +34,27 @@
 //                  on the 128-row side so no tensor-core work is padding).
 // Every mbarrier wait is bounded; on running out the kernel records
 // LMOE_ERR_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and returns.
-#include <cuda_bf16.h>
-#include <string.h>
-
-#include "lmoe_internal.h"
-#include "ptx.cuh"
-
-#ifndef LMOE_CHUNK_KB
-#define LMOE_CHUNK_KB 4   // k-blocks (of 64) per TMEM accumulation chunk
-#endif
-#ifndef LMOE_PROMOTE_F64
-#define LMOE_PROMOTE_F64 0  // 1: chunk partials are added into fp64 registers
-#endif
-#ifndef LMOE_MAX_BN
-#define LMOE_MAX_BN 256
-#endif
+#include "gemm_common.cuh"
 
 namespace lmoe {
 namespace {
 
-constexpr int kMaxMaps = 8;
-constexpr int kGroupM = 16;
-
-struct alignas(64) TcParams {
-    CUtensorMap maps[kMaxMaps];
-    GemmProblem prob[2];
-    int nprob;
-    int nmaps;
-    int dense_tiles[2];
-    DeviceRouting r;
-    int* err;
-    unsigned spin;
-};
-
-struct TileInfo {
-    int p;       // problem
-    int row0;    // first activation row (permuted row for grouped problems)
-    int rows;    // valid activation rows in this tile
-    int wrow0;   // first weight row (row of B)
-    int col0;    // first output column
-    int e;       // expert of a grouped tile (-1 for dense problems)
-    bool half;   // non-swapped tile with <= 64 valid rows: M = 64 MMAs (the expert's ragged tail)
-};
-
-template <int BN, bool kSwap, bool kFp4 = false>
-struct Shape {
-    static constexpr int XR = 128;            // rows of the MMA A operand tile
-    static constexpr int YR = BN;             // rows of the MMA B operand tile
-    static constexpr int kXBytes = XR * kBK * 2;
-    static constexpr int kYBytes = YR * kBK * 2;
-    static constexpr int kStageBytes = kXBytes + kYBytes;
-    static constexpr int kActRows = kSwap ? BN : 128;   // activation rows per tile
-    static constexpr int kOutCols = kSwap ? 128 : BN;   // output columns per tile
-    // K is accumulated in chunks of kChunkKB k-blocks in TMEM; each chunk is
-    // added into fp32 registers by the epilogue (see the file comment).
-    static constexpr int kChunkKB = LMOE_CHUNK_KB;
-    static constexpr int kBufs = (4 * BN <= 512) ? 4 : 512 / BN;     // TMEM chunk buffers
-    static constexpr int kCols = kBufs * BN;
-    static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
-                                        : kCols <= 256 ? 256 : 512;
-    static constexpr int kEpiWarps = BN >= 128 ? 8 : 4;  // two warps per TMEM lane quarter for wide tiles
-    static constexpr int kColsPerThread = BN / (kEpiWarps / 4);
-    // NVFP4 weights (swap tiles): the 128 x 64 weight tile arrives as 4096 bytes of
-    // E2M1 codes and 512 bytes of E4M3 scales, and dequantisation warps write the
-    // bf16 operand tile from them.
-    static constexpr int kRawBytes = kFp4 ? 4096 + 512 : 0;
-    static constexpr int kTxBytes = kFp4 ? kRawBytes + kYBytes : kStageBytes;  // bytes the producer's copies carry
-    // Dequantisation warps, in groups that take alternate k-blocks so that
-    // several stages convert at once: 8 groups of 1 warp for decode tiles,
-    // 2 groups of 2 warps where the registers allow fewer warps.
-    static constexpr int kDeqWarps = !kFp4 ? 0 : BN <= 64 ? 8 : 4;
-    static constexpr int kDeqGroups = !kFp4 ? 1 : BN <= 64 ? 8 : 2;
-    static constexpr int kDeqGroupWarps = kFp4 ? kDeqWarps / kDeqGroups : 1;
-    static constexpr int kDeqItems = kFp4 ? 256 / (32 * kDeqGroupWarps) : 0;  // (row, half-row) items per thread
-    static constexpr int kThreads = 64 + 32 * (kEpiWarps + kDeqWarps);
-    // per epilogue warp: one 32-row x 128-byte output box, 128-byte swizzled, for bulk tensor stores
-    static constexpr int kStageOutBytes = kSwap ? 0 : 4096;
-    static constexpr int kBarBytes = 512;
-    static constexpr int kLutBytes = kFp4 ? 256 * 4 : 0;
-    static_assert(!kFp4 || kSwap, "NVFP4 weights sit on the MMA M side");
-};
-
-// Per-expert tile prefix and tile records of a grouped problem for activation
-// tiles of R rows.
-template <int R>
-__device__ __forceinline__ const int* grouped_prefix(const DeviceRouting& r) {
-    static_assert(R == 32 || R == 64 || R == 128 || R == 256, "activation tile rows");
-    return R == kDecodeTN ? r.pfxdec : R == 64 ? r.pfx64 : R == 128 ? r.pfx128 : r.pfx256;
-}
-template <int R>
-__device__ __forceinline__ const int4* grouped_records(const DeviceRouting& r) {
-    return R == kDecodeTN ? r.rec32 : R == 64 ? r.rec64 : R == 128 ? r.rec128 : r.rec256;
-}
-
-__device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
-
-template <int BN, bool kSwap>
-__device__ __forceinline__ int total_tiles(const TcParams& P) {
+template <int BN, int STAGES, bool kSwap>
+__global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
     using S = Shape<BN, kSwap>;
-    if (P.prob[0].grouped) {
-        const int* pfx = grouped_prefix<S::kActRows>(P.r);
-        return pfx[P.r.E] * n_col_tiles(P.prob[0], S::kOutCols);
-    }
-    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
-}
-
-// Tile t -> coordinates. Dense problems are rasterised in groups of kGroupM
-// row tiles (column tiles outer within a group) so that concurrently running
-// CTAs share both operands in L2. Grouped problems walk experts in order,
-// column tiles inner, so an expert's weights are read while its rows are hot;
-// their row tiles come from the permutation's tile records (one 16-byte load,
-// instead of a dependent search over the per-expert prefix at every tile).
-template <int BN, bool kSwap>
-__device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
-    using S = Shape<BN, kSwap>;
-    TileInfo ti;
-    if (P.prob[0].grouped) {
-        const GemmProblem& pr = P.prob[0];
-        const int nct = n_col_tiles(pr, S::kOutCols);
-        const int mt = t / nct, ct = t % nct;
-        const int4 rc = __ldg(grouped_records<S::kActRows>(P.r) + mt);
-        const int e = rc.x;
-        ti.p = 0;
-        ti.row0 = rc.y;
-        ti.rows = rc.z;
-        ti.col0 = ct * S::kOutCols;
-        ti.wrow0 = e * pr.b_rows_per_expert + ti.col0;
-        ti.e = e;
-        ti.half = !kSwap && ti.rows <= 64;
-        return ti;
-    }
-    int p = 0;
-    if (P.nprob > 1 && t >= P.dense_tiles[0]) {
-        t -= P.dense_tiles[0];
-        p = 1;
-    }
-    const GemmProblem& pr = P.prob[p];
-    const int nct = n_col_tiles(pr, S::kOutCols);
-    const int mtc = (pr.m_rows + S::kActRows - 1) / S::kActRows;
-    int mt, ct;
-    if (kSwap) {  // token tiles inner: the tiles that share a weight block run together
-        ct = t / mtc;
-        mt = t % mtc;
-    } else {
-        const int g = t / (kGroupM * nct), r = t % (kGroupM * nct);
-        const int ms = min(kGroupM, mtc - g * kGroupM);
-        mt = g * kGroupM + r % ms;
-        ct = r / ms;
-    }
-    ti.p = p;
-    ti.row0 = mt * S::kActRows;
-    ti.rows = min(S::kActRows, pr.m_rows - ti.row0);
-    ti.col0 = ct * S::kOutCols;
-    ti.wrow0 = ti.col0;
-    ti.e = -1;
-    ti.half = !kSwap && ti.rows <= 64;
-    return ti;
-}
-
-// Epilogue of one tile from the thread's fp32 accumulators acc[CW], which
-// hold accumulator columns c0 .. c0+CW-1 of TMEM lane `lane_row`.
-// Non-swapped tiles with an output tensor map are written with bulk tensor
-// stores: the warp stages its 32 rows x 128 bytes in shared memory with the
-// 128-byte swizzle (conflict-free writes) and one lane issues the store. Rows
-// past a dense problem's end are clipped by the tensor bounds; a grouped tile
-// whose 32-row slab runs into the next expert's rows uses plain masked stores.
-template <int BN, bool kSwap, int CW>
-__device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const TileInfo& ti, int lane_row, int c0,
-                                               float (&acc)[CW], const CUtensorMap* omap, uint8_t* stage) {
-    const int epi = pr.epi;
-    const int lane = threadIdx.x & 31;
-    if (pr.wscale) {  // NVFP4 experts: h = g_e * (sum of code * block scale * activation)
-        const float g = __ldg(&pr.wscale[ti.e]);
-#pragma unroll
-        for (int i = 0; i < CW; ++i) acc[i] *= g;
-    }
-    if (epi == EPI_RELU2_BF16 || epi == EPI_RELU2_F32) {
-#pragma unroll
-        for (int i = 0; i < CW; ++i) {
-            float a = fmaxf(acc[i], 0.f);
-            acc[i] = a * a;
-        }
-    }
-    if (!kSwap && pr.resid && lane_row < ti.rows) {  // block residual: out = resid + acc (fp32)
-        const uint4* rs = reinterpret_cast<const uint4*>(pr.resid + (size_t)(ti.row0 + lane_row) * pr.ldo + ti.col0 + c0);
-#pragma unroll
-        for (int q8 = 0; q8 < CW / 8; ++q8) {
-            const uint4 u = __ldg(rs + q8);
-            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc[q8 * 8 + 2 * j] += __uint_as_float(w4[j] << 16);
-                acc[q8 * 8 + 2 * j + 1] += __uint_as_float(w4[j] & 0xFFFF0000u);
-            }
-        }
-    }
-    if (!kSwap) {
-        const bool bf16_out = epi == EPI_BF16 || epi == EPI_RELU2_BF16;
-        const int slab0 = lane_row - lane;  // first row of this warp's 32-row slab
-        if (omap && (!pr.grouped || slab0 + 32 <= ti.rows)) {
-            if (epi == EPI_SCALE_F32) {
-                const float sc = __ldg(&pr.row_scale[ti.row0 + lane_row]);
-#pragma unroll
-                for (int i = 0; i < CW; ++i) acc[i] *= sc;
-            }
-            uint8_t* myrow = stage + lane * 128;
-            constexpr int kGroupsF32 = CW / 32, kGroupsBf16 = CW / 64;
-            const int ngroups = bf16_out ? kGroupsBf16 : kGroupsF32;
-#pragma unroll
-            for (int g = 0; g < (CW / 32); ++g) {
-                if (g >= ngroups) break;
-                if (lane == 0) bulk_wait_read_all();  // staging buffer free again
-                __syncwarp();
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v;
-                    if (bf16_out) {
-                        const int b = g * 64 + c * 8;
-                        v = make_uint4(pack_bf16x2(acc[b], acc[b + 1]), pack_bf16x2(acc[b + 2], acc[b + 3]),
-                                       pack_bf16x2(acc[b + 4], acc[b + 5]), pack_bf16x2(acc[b + 6], acc[b + 7]));
-                    } else {
-                        const int b = g * 32 + c * 4;
-                        v = make_uint4(__float_as_uint(acc[b]), __float_as_uint(acc[b + 1]),
-                                       __float_as_uint(acc[b + 2]), __float_as_uint(acc[b + 3]));
-                    }
-                    *reinterpret_cast<uint4*>(myrow + ((c ^ (lane & 7)) << 4)) = v;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const int x = ti.col0 + c0 + g * (bf16_out ? 64 : 32);
-                    tma_store_2d(omap, stage, x, ti.row0 + slab0);
-                    bulk_commit();
-                }
-            }
-            return;
-        }
-        // thread owns activation row (row0 + lane_row), output columns col0 + c0 ..
-        if (lane_row >= ti.rows) return;
-        const long long row = ti.row0 + lane_row;
-        if (epi == EPI_SCALE_F32) {
-            const float sc = __ldg(&pr.row_scale[row]);
-#pragma unroll
-            for (int i = 0; i < CW; ++i) acc[i] *= sc;
-        }
-        if (bf16_out) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) + row * pr.ldo + ti.col0 + c0);
-#pragma unroll
-            for (int q = 0; q < CW / 8; ++q)
-                dst[q] = make_uint4(pack_bf16x2(acc[8 * q], acc[8 * q + 1]), pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]),
-                                    pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]),
-                                    pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
-        } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + row * pr.ldo + ti.col0 + c0);
-#pragma unroll
-            for (int q = 0; q < CW / 4; ++q)
-                dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-        }
-    } else {
-        // thread owns output column (col0 + lane_row); accumulator columns are
-        // the tile's tokens row0 + c0 + i. Lanes write consecutive columns.
-        const long long col = ti.col0 + lane_row;
-#pragma unroll
-        for (int i = 0; i < CW; ++i) {
-            const int tok = c0 + i;
-            if (tok < ti.rows) {
-                const long long row = ti.row0 + tok;
-                float x = acc[i];
-                if (epi == EPI_SCALE_F32) x *= __ldg(&pr.row_scale[row]);
-                if (pr.resid) x += __uint_as_float((uint32_t)pr.resid[row * pr.ldo + col] << 16);
-                if (epi == EPI_BF16 || epi == EPI_RELU2_BF16)
-                    static_cast<__nv_bfloat16*>(pr.out)[row * pr.ldo + col] = __float2bfloat16_rn(x);
-                else
-                    static_cast<float*>(pr.out)[row * pr.ldo + col] = x;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ int tile_kblocks(const GemmProblem& pr) {
-    int n = pr.kdim[0] / kBK;
-    if (pr.nseg > 1) n += pr.kdim[1] / kBK;
-    return n;
-}
-
-// ---------------------------------------------------------------- NVFP4
-// E2M1 codes -> bf16. Eight codes (one 32-bit word, element i in nibble i) give
-// four bf16 pairs. The three magnitude bits index two byte tables held in
-// registers (high and low byte of the bf16 value of 0, 0.5, 1, 1.5, 2, 3, 4, 6)
-// with byte permutes; the sign bits are moved to bit 7 of the high bytes; the
-// block scale (bf16, both halves) multiplies the pair. code * scale has at most
-// 6 significant bits and lies in [2^-10, 2688], so the product is exact.
-__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t c, uint32_t scale2) {
-    constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;  // high bytes of magnitudes 0..3, 4..7
-    constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;  // low bytes
-    const uint32_t mag = c & 0x77777777u;
-    const uint32_t d = c << 4;  // bit 7 of byte j = sign of element 2j; bit 7 of c's byte j = sign of 2j + 1
-    const uint32_t mhi = mag >> 16;
-    const uint32_t h0 = prmt(kHi0, kHi1, mag) | (prmt(d, c, 0x5140u) & 0x80808080u);
-    const uint32_t l0 = prmt(kLo0, kLo1, mag);
-    const uint32_t h1 = prmt(kHi0, kHi1, mhi) | (prmt(d, c, 0x7362u) & 0x80808080u);
-    const uint32_t l1 = prmt(kLo0, kLo1, mhi);
-    uint4 o;
-    o.x = mul_bf16x2(prmt(l0, h0, 0x5140u), scale2);
-    o.y = mul_bf16x2(prmt(l0, h0, 0x7362u), scale2);
-    o.z = mul_bf16x2(prmt(l1, h1, 0x5140u), scale2);
-    o.w = mul_bf16x2(prmt(l1, h1, 0x7362u), scale2);
-    return o;
-}
-
-// bf16 value of an E4M3 byte (bias 7, 3 mantissa bits, subnormals m * 2^-9),
-// duplicated in both halves. Exact: E4M3 values need 4 significant bits.
-__device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
-    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-    float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
-    if (b & 0x80u) v = -v;
-    const uint32_t h = __float_as_uint(v) >> 16;
-    return h | (h << 16);
-}
-
-template <int BN, int STAGES, bool kSwap, bool kFp4 = false>
-__global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
-    using S = Shape<BN, kSwap, kFp4>;
     constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
     uint8_t* sX = smem;                                  // STAGES x kXBytes
     uint8_t* sY = smem + STAGES * S::kXBytes;            // STAGES x kYBytes
-    uint8_t* sRaw = sY + STAGES * S::kYBytes;            // STAGES x kRawBytes (NVFP4 codes + scales)
-    uint8_t* sOut = sRaw + STAGES * S::kRawBytes;        // kEpiWarps x kStageOutBytes
+    uint8_t* sOut = sY + STAGES * S::kYBytes;            // kEpiWarps x kStageOutBytes
     uint64_t* full = reinterpret_cast<uint64_t*>(sOut + S::kEpiWarps * S::kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* cfull = empty + STAGES;   // chunk accumulator ready (MMA -> epilogue)
     uint64_t* cempty = cfull + NB;      // chunk accumulator drained (epilogue -> MMA)
     uint64_t* done = cempty + NB;
-    uint64_t* deq = done + 1;           // NVFP4: bf16 weight tile written (dequantisation -> MMA)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(deq + STAGES);
-    uint32_t* scale_lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(full) + S::kBarBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -384,13 +67,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc
             mbar_init(&cempty[b], S::kEpiWarps);
         }
         mbar_init(done, 1);
-        if (kFp4)
-            for (int s = 0; s < STAGES; ++s) mbar_init(&deq[s], S::kDeqGroupWarps);
         fence_mbar_init();
     }
-    if (kFp4 && warp >= 2 + S::kEpiWarps)
-        for (int b = threadIdx.x - 32 * (2 + S::kEpiWarps); b < 256; b += 32 * S::kDeqWarps)
-            scale_lut[b] = e4m3_to_bf16x2((uint32_t)b);
     if (warp == 0 && lane == 0)
         for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
     if (warp == 1) {
@@ -421,15 +99,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
-                    if (kFp4) {
-                        // weight tile (128 rows x 64 K) of NVFP4 codes and scales; tokens by TMA
-                        const long long tile = (long long)(ti.wrow0 >> 7) * kb_n + kb;
-                        uint8_t* raw = sRaw + stage * S::kRawBytes;
-                        bulk_load(raw, pr.wq_codes + tile * 4096, 4096, &full[stage]);
-                        bulk_load(raw + 4096, pr.wq_sf + tile * 512, 512, &full[stage]);
-                        tma_load_2d(sY + stage * S::kYBytes, amap, &full[stage], kb * kBK, ti.row0);
-                    } else if (!kSwap) {
+                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    if (!kSwap) {
                         tma_load_2d(sX + stage * S::kXBytes, amap, &full[stage], kb * kBK, ti.row0);
                         tma_load_2d(sY + stage * S::kYBytes, bmap, &full[stage], kb * kBK, ti.wrow0);
                     } else {
@@ -470,7 +141,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc
                 const uint32_t d = tmem_base + (uint32_t)(buf * BN);
                 const int kb1 = min(kb_total, kb0 + CK);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait_bounded(kFp4 ? &deq[stage] : &full[stage], phase, P.spin, err)) {
+                    if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
                         ok = false;
                         break;
                     }
@@ -500,64 +171,6 @@ __global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc
         // all MMAs issued by this thread have completed before TMEM is freed
         umma_commit(done);
         mbar_wait_bounded(done, 0, 1u << 26, err);
-    } else if (kFp4 && warp >= 2 + S::kEpiWarps) {
-        // ------------------------------------------------ NVFP4 dequantisation
-        // Each thread converts (row, half-row) items of the 128 x 64 weight tile:
-        // 32 codes (16 bytes) and their two block scales -> four 16-byte chunks
-        // of the 128-byte-swizzled bf16 operand row (chunk j at (j ^ (row & 7)) * 16).
-        // Group g takes the k-blocks c with c % kDeqGroups == g (c counts the
-        // CTA's k-blocks in the producer's order), so groups convert different
-        // stages at the same time.
-        const int dw = warp - (2 + S::kEpiWarps);
-        const int grp = dw / S::kDeqGroupWarps;
-        const int gt = (dw % S::kDeqGroupWarps) * 32 + lane;  // thread within the group
-        uint32_t c = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const TileInfo ti = decode_tile<BN, kSwap>(P, t);
-            const int kb_total = tile_kblocks(P.prob[ti.p]);
-            for (int kb = 0; kb < kb_total; ++kb, ++c) {
-                if ((int)(c % S::kDeqGroups) != grp) continue;
-                const int stage = (int)(c % STAGES);
-                const uint32_t phase = (c / STAGES) & 1u;
-                if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* raw = sRaw + stage * S::kRawBytes;
-                uint8_t* dst = sX + stage * S::kXBytes;
-                constexpr int NI = S::kDeqItems > 0 ? S::kDeqItems : 1;  // (the branch is dead without NVFP4)
-#pragma unroll
-                for (int i0 = 0; i0 < NI; i0 += 2) {  // two items' loads first, so their conversions overlap
-                    constexpr int NJ = NI >= 2 ? 2 : 1;
-                    uint4 cw[NJ];
-                    uint32_t sA[NJ], sB[NJ];
-#pragma unroll
-                    for (int j = 0; j < NJ; ++j) {
-                        const int it = gt + (i0 + j) * 32 * S::kDeqGroupWarps, r = it >> 1, hh = it & 1;
-                        cw[j] = *reinterpret_cast<const uint4*>(raw + r * 32 + hh * 16);
-                        const uint32_t sb = *reinterpret_cast<const uint16_t*>(raw + 4096 + r * 4 + hh * 2);
-                        sA[j] = scale_lut[sb & 0xFFu];
-                        sB[j] = scale_lut[sb >> 8];
-                    }
-#pragma unroll
-                    for (int j = 0; j < NJ; ++j) {
-                        const int it = gt + (i0 + j) * 32 * S::kDeqGroupWarps, r = it >> 1, hh = it & 1;
-                        uint8_t* row = dst + r * 128;
-                        const int sw = r & 7, j0 = 4 * hh;
-                        const uint4 o0 = e2m1x8_to_bf16(cw[j].x, sA[j]), o1 = e2m1x8_to_bf16(cw[j].y, sA[j]);
-                        const uint4 o2 = e2m1x8_to_bf16(cw[j].z, sB[j]), o3 = e2m1x8_to_bf16(cw[j].w, sB[j]);
-                        st_shared_v4(row + (((j0 + 0) ^ sw) << 4), o0);
-                        st_shared_v4(row + (((j0 + 1) ^ sw) << 4), o1);
-                        st_shared_v4(row + (((j0 + 2) ^ sw) << 4), o2);
-                        st_shared_v4(row + (((j0 + 3) ^ sw) << 4), o3);
-                    }
-                }
-                fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&deq[stage]);
-            }
-        }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
         const int ew = warp - 2;
@@ -638,8 +251,9 @@ __global__ void __launch_bounds__(Shape<BN, kSwap, kFp4>::kThreads, 1) k_gemm_tc
 }
 
 // ---------------------------------------------------------------- 2-SM pairs
-// (Selected with LMOE_OPT_GEMM_PATH = 4; measured no faster than the single-SM
-// tiles on this layer, whose steady state is set by the 1 kW power cap.)
+// (Selected with LMOE_OPT_GEMM_PATH = 4. Slower than the single-SM tiles on
+// this layer at its power-capped steady state: 25.7 against 23.4-23.9 ms per
+// 16384-token Ultra forward, each path timed in its own process.)
 // A cluster of two CTAs on neighbouring SMs computes one 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M = 256, N = 256). Each CTA stages its own 128 A
 // rows and its own half (128 rows) of B, 32 KB per k-block instead of the
@@ -892,23 +506,22 @@ __global__ void __launch_bounds__(PairShape::kThreads, 1) k_gemm_tc_pair(const _
     if (warp == 1) tmem_dealloc_pair(tmem_base, S::kTmemCols);
 }
 
-template <int BN, int STAGES, bool kSwap, bool kFp4>
+template <int BN, int STAGES, bool kSwap>
 constexpr size_t smem_bytes() {
-    using S = Shape<BN, kSwap, kFp4>;
-    return 1024 + (size_t)STAGES * (S::kStageBytes + S::kRawBytes) + (size_t)S::kEpiWarps * S::kStageOutBytes +
-           S::kBarBytes + S::kLutBytes;
+    using S = Shape<BN, kSwap>;
+    return 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 512;
 }
 
-template <int BN, int STAGES, bool kSwap, bool kFp4 = false>
+template <int BN, int STAGES, bool kSwap>
 cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
-    using S = Shape<BN, kSwap, kFp4>;
-    constexpr size_t smem = smem_bytes<BN, STAGES, kSwap, kFp4>();
+    using S = Shape<BN, kSwap>;
+    constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
     static_assert(smem <= 232448, "shared memory");
-    static_assert((3 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= S::kBarBytes, "barrier area");
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap, kFp4>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 512, "barrier area");
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    k_gemm_tc<BN, STAGES, kSwap, kFp4><<<grid, S::kThreads, smem, s>>>(P);
+    k_gemm_tc<BN, STAGES, kSwap><<<grid, S::kThreads, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -924,18 +537,6 @@ int tc_num_sms() {
         g_num_sms = n > 0 ? n : 148;
     }
     return g_num_sms;
-}
-
-static void fill_params(TcParams& P, const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
-                        const DeviceRouting& r, int* err, unsigned spin) {
-    memset(&P, 0, sizeof(P));
-    for (int i = 0; i < nmaps && i < kMaxMaps; ++i) P.maps[i] = maps[i];
-    for (int i = 0; i < nprob; ++i) P.prob[i] = probs[i];
-    P.nprob = nprob;
-    P.nmaps = nmaps < kMaxMaps ? nmaps : kMaxMaps;
-    P.r = r;
-    P.err = err;
-    P.spin = spin;
 }
 
 // Dense tile counts (host side) and a grid no larger than the work.
@@ -976,7 +577,7 @@ cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmPr
     using S = PairShape;
     constexpr size_t smem = 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 256;
     static_assert(smem <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 256, "barrier area");
+    static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 512, "barrier area");
     TcParams P;
     fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
     int pairs = tc_num_sms() / 2;
@@ -1023,22 +624,6 @@ cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const Gemm
         if (grid < 1) return cudaSuccess;
     }
     return launch_impl<kDecodeTN, 10, true>(P, grid, s);
-}
-
-// Grouped expert GEMMs with NVFP4 weights: weight-stationary tiles (128 weight
-// rows on the MMA M side), bn = 32 tokens per tile (decode) or 128 (prefill).
-cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
-                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
-    if (nprob != 1 || !probs[0].grouped || probs[0].nseg != 1 || !probs[0].wq_codes || !probs[0].wq_sf)
-        return cudaErrorInvalidValue;
-    TcParams P;
-    fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
-    const int grid = tc_num_sms();
-    switch (bn) {
-        case kDecodeTN: return launch_impl<kDecodeTN, 8, true, true>(P, grid, s);
-        case 128: return launch_impl<128, 6, true, true>(P, grid, s);
-        default: return cudaErrorInvalidValue;
-    }
 }
 
 // ---------------------------------------------------------------- self-test

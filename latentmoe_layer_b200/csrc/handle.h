@@ -13,6 +13,7 @@ struct lmoe_handle {
     unsigned spin_limit = 1u << 24;
     int num_sms = 148;
     int launches = 0;                  // kernels launched by the last call
+    int last_cuda_error = 0;           // cudaError_t of the last runtime call that failed (0: none yet)
     void* const* prof_events = nullptr;  // latentmoe_set_profile_events
     int prof_n = 0;
 };

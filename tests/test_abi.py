@@ -163,3 +163,27 @@ def test_bounded_wait_times_out_and_context_survives(lib):
     torch.cuda.synchronize()
     assert torch.isfinite(y).all()
     assert layer.stats().device_error == 0
+
+
+
+@pytest.mark.gpu
+def test_profile_events_must_exist(lib):
+    # a NULL event (e.g. a framework event never recorded, hence not created yet) is refused;
+    # created events are accepted and a forward with them succeeds
+    import torch
+    import helpers as H
+    layer, dev = H.device_layer(synth.TINY, max_tokens=64)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    unrecorded = (ctypes.c_void_p * 8)(*[e.cuda_event for e in evs])
+    assert lm.latentmoe_set_profile_events(layer.h, ctypes.cast(unrecorded, ctypes.c_void_p), 8) == \
+        lm.LMOE_ERR_INVALID_ARG
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    created = (ctypes.c_void_p * 8)(*[e.cuda_event for e in evs])
+    assert lm.latentmoe_set_profile_events(layer.h, ctypes.cast(created, ctypes.c_void_p), 8) == lm.LMOE_OK
+    layer.forward(dev["x"])
+    torch.cuda.synchronize()
+    assert evs[0].elapsed_time(evs[7]) > 0
+    assert lm.latentmoe_set_profile_events(layer.h, None, 0) == lm.LMOE_OK
+    layer.close()
