@@ -10,7 +10,7 @@
 #include "ptx.cuh"
 
 #ifndef LMOE_CHUNK_KB
-#define LMOE_CHUNK_KB 4   // k-blocks (of 64) per TMEM accumulation chunk
+#define LMOE_CHUNK_KB 8   // k-blocks (of 64) per TMEM accumulation chunk
 #endif
 #ifndef LMOE_PROMOTE_F64
 #define LMOE_PROMOTE_F64 0  // 1: chunk partials are added into fp64 registers
