@@ -9,15 +9,16 @@
 // is that of the bf16 path applied to the dequantised weights.
 //
 // Weight-stationary tiles: MMA M = 128 weight rows, N = BN tokens of one
-// expert (BN = 32 at decode sizes, 128 otherwise). One ring of stages, each
-// holding KB k-blocks of 64: the token tiles (TMA, 128-byte swizzle), the
-// codes and scales (bulk copies), and the bf16 weight tiles the
-// dequantisation warps write from them. Every barrier wait and commit sits on
-// the path of a 32-token tile, whose tensor-core work per k-block is short,
-// so a stage carries several k-blocks to spread that cost.
+// expert (BN = 32 at decode sizes, 128 otherwise). A ring of shared-memory
+// stages, each holding KB k-blocks of 64 (token tiles by TMA with the 128-byte
+// swizzle, codes and scales by bulk copy), feeds dequantisation warps that
+// write the bf16 weight rows into TMEM slots; the MMA reads A from TMEM and B
+// (tokens) from shared memory. Every barrier wait and commit sits on the path
+// of a 32-token tile, whose tensor-core work per k-block is short, so a stage
+// carries several k-blocks to spread that cost.
 // Roles: warp 0 producer, warp 1 MMA issuer and TMEM owner, then the epilogue
-// warps (TMEM chunk drains, as in the bf16 kernel), then dequantisation warps
-// in G groups that take the stages in turn.
+// warps (TMEM chunk drains, as in the bf16 kernel), then the dequantisation
+// warps.
 #include "gemm_common.cuh"
 
 namespace lmoe {
@@ -57,42 +58,57 @@ __device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
     return h | (h << 16);
 }
 
-template <int BN, int STAGES, int KB, int G>
-struct Fp4Shape {
-    using T = Shape<BN, true>;                         // TMEM ring, epilogue split, token tile rows
-    static constexpr int kTokBytes = BN * kBK * 2;     // token tile of one k-block, BN rows x 128 bytes
-    static constexpr int kOpBytes = 128 * kBK * 2;     // bf16 weight tile of one k-block
-    // stage: KB token tiles | KB bf16 weight tiles | KB x 4096 code bytes | KB x 512 scale bytes
-    static constexpr int kOffOp = KB * kTokBytes;
-    static constexpr int kOffCodes = kOffOp + KB * kOpBytes;
+// ------------------------------------------------------------------------------
+// The dequantised weights live in TMEM: the tensor core takes its A operand
+// (128 weight rows x K) from TMEM, so the bf16 weight tile never passes through
+// shared memory (with it in shared memory, the codes read, the bf16 tile
+// written and read back, and the copies made ~49 KB of shared-memory traffic
+// per k-block; now ~17 KB). Each
+// dequantisation thread owns one weight row = one TMEM lane: it reads the row's
+// 32 code bytes and 4 scale bytes and stores 32 columns (64 bf16) with
+// tcgen05.st. A warp may only touch its own TMEM lane quarter, so the
+// dequantisation warps form G groups of four (one per quarter); every group
+// works on every stage, group g converting the stage's k-blocks j with
+// j % G == g, so a stage's conversion is spread over all G x 4 warps (one
+// group per stage made each stage a long serial chain per thread).
+// TMEM columns: [0, 256) accumulator chunk buffers, [256, 512)
+// AS slots of KB bf16 weight tiles. The shared-memory ring (codes, scales,
+// token tiles) is deeper than the slot ring, so copies run far ahead of the
+// conversions: before it overwrites slot c % AS, the conversion of stage c
+// waits for the MMA of stage c - AS, the slot's last reader, on that stage's
+// `empty` barrier (no barrier is added to the MMA's path).
+template <int BN, int STAGES, int KB, int G, int AS>
+struct Fp4TmShape {
+    using T = Shape<BN, true>;
+    static constexpr int kTokBytes = BN * kBK * 2;
+    static constexpr int kOffCodes = KB * kTokBytes;
     static constexpr int kOffSf = kOffCodes + KB * 4096;
-    static constexpr int kStageBytes = (kOffSf + KB * 512 + 1023) & ~1023;  // swizzled tiles stay 1024-aligned
-    static constexpr int kTxBytes = KB * (kTokBytes + 4096 + 512);          // bytes the producer's copies carry
-    static constexpr int kDeqWarps = BN <= 64 ? 8 : 4;
-    static constexpr int kGroupWarps = kDeqWarps / G;
-    static constexpr int kItems = KB * 256 / (32 * kGroupWarps);  // (row, half-row) items per thread and stage
+    static constexpr int kStageBytes = (kOffSf + KB * 512 + 1023) & ~1023;
+    static constexpr int kTxBytes = KB * (kTokBytes + 4096 + 512);
+    static constexpr int kBufs = 256 / BN;           // accumulator chunk buffers in columns [0, 256)
+    static constexpr uint32_t kColA = 256;           // first column of the weight tiles
+    static constexpr int kDeqWarps = 4 * G;
     static constexpr int kThreads = 64 + 32 * (T::kEpiWarps + kDeqWarps);
     static constexpr int kBarBytes = 1024;
-    static constexpr int kBars = 3 * STAGES + 2 * T::kBufs + 1;
+    static constexpr int kBars = 3 * STAGES + 2 * kBufs + 1;
     static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStageBytes + kBarBytes + 1024;
+    static_assert(AS * KB * 32 <= 256 && AS <= STAGES, "weight tiles fit TMEM columns [256, 512)");
     static_assert(kBars * 8 + 4 <= kBarBytes, "barrier area");
-    static_assert(kDeqWarps % G == 0 && G <= STAGES && kItems % 2 == 0, "dequantisation groups");
-    static_assert(T::kChunkKB % KB == 0, "a chunk is whole stages");
-    static_assert(kSmem <= 232448, "shared memory");
-    static_assert(STAGES <= 32, "issued-load mask");
+    static_assert(KB % G == 0 && T::kChunkKB % KB == 0, "groups / chunks");
+    static_assert(kSmem <= 232448 && STAGES <= 32, "shared memory");
 };
 
-template <int BN, int STAGES, int KB, int G>
-__global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
-    k_gemm_nvfp4(const __grid_constant__ TcParams P) {
-    using F = Fp4Shape<BN, STAGES, KB, G>;
+template <int BN, int STAGES, int KB, int G, int AS>
+__global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1)
+    k_gemm_nvfp4_tm(const __grid_constant__ TcParams P) {
+    using F = Fp4TmShape<BN, STAGES, KB, G, AS>;
     using S = typename F::T;
-    constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
+    constexpr int NB = F::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * F::kStageBytes);  // copies landed (producer)
-    uint64_t* deq = full + STAGES;         // bf16 weight tiles written (dequantisation -> MMA)
+    uint64_t* deq = full + STAGES;         // weight tiles stored in TMEM (dequantisation -> MMA)
     uint64_t* empty = deq + STAGES;        // MMA done with the stage (MMA -> producer)
     uint64_t* cfull = empty + STAGES;      // chunk accumulator ready (MMA -> epilogue)
     uint64_t* cempty = cfull + NB;         // chunk accumulator drained (epilogue -> MMA)
@@ -104,7 +120,7 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&deq[s], F::kGroupWarps);
+            mbar_init(&deq[s], 4 * G);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < NB; ++b) {
@@ -120,7 +136,7 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
     if (warp == 0 && lane == 0)
         for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
     if (warp == 1) {
-        tmem_alloc(tmem_slot, S::kTmemCols);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -159,7 +175,6 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
                 issued_par = (issued_par & ~(1u << s)) | (ph << s);
             }
         }
-        // every copy this thread issued has landed before the CTA can exit
         for (int s = 0; s < STAGES; ++s)
             if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
     } else if (warp == 1 && lane == 0) {
@@ -179,7 +194,8 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
                 const int kb1 = min(kb_n, kb0 + CK);
                 for (int kb = kb0; kb < kb1; kb += KB, ++c) {
                     const int s = (int)(c % STAGES);
-                    if (!mbar_wait_bounded(&deq[s], (c / STAGES) & 1u, spin, err)) {
+                    if (!mbar_wait_bounded(&deq[s], (c / STAGES) & 1u, spin, err) ||
+                        !mbar_wait_bounded(&full[s], (c / STAGES) & 1u, spin, err)) {
                         ok = false;
                         break;
                     }
@@ -187,12 +203,12 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
                     const uint8_t* st = smem + s * F::kStageBytes;
 #pragma unroll
                     for (int j = 0; j < KB; ++j) {
-                        const uint64_t adesc = sdesc_sw128(smem_u32(st + F::kOffOp + j * F::kOpBytes));
+                        const uint32_t a = tmem_base + F::kColA + (uint32_t)(((c % AS) * KB + j) * 32);
                         const uint64_t bdesc = sdesc_sw128(smem_u32(st + j * F::kTokBytes));
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk)
-                            umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
-                                      (kb + j > kb0 || kk > 0) ? 1u : 0u);
+                            umma_bf16_tmem_a(d, a + (uint32_t)(kk * 8), bdesc + (uint64_t)(kk * 2), idesc,
+                                             (kb + j > kb0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -207,55 +223,55 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
         umma_commit(done);
         mbar_wait_bounded(done, 0, 1u << 26, err);
     } else if (warp >= dq0) {
-        // ------------------------------------------------ dequantisation
-        // Group g converts the stages c with c % G == g (c counts the CTA's
-        // stages in the producer's order). A thread converts (row, half-row)
-        // items: 32 codes (16 bytes) and their two block scales -> four 16-byte
-        // chunks of the 128-byte-swizzled bf16 row (chunk j at (j ^ (row & 7)) * 16).
-        // Item it of a stage: k-block it / 256 of the stage, row (it % 256) / 2.
+        // ------------------------------------------------ dequantisation into TMEM
         const int dw = warp - dq0;
-        const int grp = dw / F::kGroupWarps;
-        const int gt = (dw % F::kGroupWarps) * 32 + lane;
+        const int grp = dw >> 2;
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;          // weight row = TMEM lane
         uint32_t c = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             for (int kb = 0; kb < kb_n; kb += KB, ++c) {
-                if ((int)(c % G) != grp) continue;
                 const int s = (int)(c % STAGES);
+                const uint32_t slot = c % AS;
+                if (c >= (uint32_t)AS) {  // the slot's last reader, the MMA of stage c - AS, has completed
+                    const uint32_t p = c - AS;
+                    if (!mbar_wait_bounded(&empty[p % STAGES], (p / STAGES) & 1u, spin, err)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 if (!mbar_wait_bounded(&full[s], (c / STAGES) & 1u, spin, err)) {
                     ok = false;
                     break;
                 }
-                uint8_t* st = smem + s * F::kStageBytes;
+                const uint8_t* st = smem + s * F::kStageBytes;
 #pragma unroll
-                for (int i0 = 0; i0 < F::kItems; i0 += 2) {  // two items' loads first, so their conversions overlap
-                    uint4 cw[2];
-                    uint32_t sA[2], sB[2];
+                for (int j = grp; j < KB; j += G) {
+                    const uint8_t* codes = st + F::kOffCodes + j * 4096 + row * 32;
+                    const uint4 c0 = ld_shared_v4(codes), c1 = ld_shared_v4(codes + 16);
+                    const uint32_t sb = ld_shared_u32(st + F::kOffSf + j * 512 + row * 4);
+                    const uint32_t s0 = ld_shared_u32(scale_lut + (sb & 0xFFu));
+                    const uint32_t s1 = ld_shared_u32(scale_lut + ((sb >> 8) & 0xFFu));
+                    const uint32_t s2 = ld_shared_u32(scale_lut + ((sb >> 16) & 0xFFu));
+                    const uint32_t s3 = ld_shared_u32(scale_lut + (sb >> 24));
+                    uint32_t w[32];
+                    const uint4 o0 = e2m1x8_to_bf16(c0.x, s0), o1 = e2m1x8_to_bf16(c0.y, s0);
+                    const uint4 o2 = e2m1x8_to_bf16(c0.z, s1), o3 = e2m1x8_to_bf16(c0.w, s1);
+                    const uint4 o4 = e2m1x8_to_bf16(c1.x, s2), o5 = e2m1x8_to_bf16(c1.y, s2);
+                    const uint4 o6 = e2m1x8_to_bf16(c1.z, s3), o7 = e2m1x8_to_bf16(c1.w, s3);
+                    const uint4 os[8] = {o0, o1, o2, o3, o4, o5, o6, o7};
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int it = gt + (i0 + j) * 32 * F::kGroupWarps, kq = it >> 8, row = (it & 255) >> 1,
-                                  hh = it & 1;
-                        const uint8_t* codes = st + F::kOffCodes + kq * 4096;
-                        cw[j] = ld_shared_v4(codes + row * 32 + hh * 16);
-                        const uint32_t sb = ld_shared_u16(st + F::kOffSf + kq * 512 + row * 4 + hh * 2);
-                        sA[j] = ld_shared_u32(scale_lut + (sb & 0xFFu));
-                        sB[j] = ld_shared_u32(scale_lut + (sb >> 8));
+                    for (int i = 0; i < 8; ++i) {
+                        w[4 * i] = os[i].x;
+                        w[4 * i + 1] = os[i].y;
+                        w[4 * i + 2] = os[i].z;
+                        w[4 * i + 3] = os[i].w;
                     }
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int it = gt + (i0 + j) * 32 * F::kGroupWarps, kq = it >> 8, row = (it & 255) >> 1,
-                                  hh = it & 1;
-                        uint8_t* drow = st + F::kOffOp + kq * F::kOpBytes + row * 128;
-                        const int sw = row & 7, j0 = 4 * hh;
-                        const uint4 o0 = e2m1x8_to_bf16(cw[j].x, sA[j]), o1 = e2m1x8_to_bf16(cw[j].y, sA[j]);
-                        const uint4 o2 = e2m1x8_to_bf16(cw[j].z, sB[j]), o3 = e2m1x8_to_bf16(cw[j].w, sB[j]);
-                        st_shared_v4(drow + (((j0 + 0) ^ sw) << 4), o0);
-                        st_shared_v4(drow + (((j0 + 1) ^ sw) << 4), o1);
-                        st_shared_v4(drow + (((j0 + 2) ^ sw) << 4), o2);
-                        st_shared_v4(drow + (((j0 + 3) ^ sw) << 4), o3);
-                    }
+                    tmem_st32(tmem_base + ((uint32_t)(q * 32) << 16) + F::kColA + (slot * KB + j) * 32u, w);
                 }
-                fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&deq[s]);
             }
@@ -264,8 +280,8 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
         // ------------------------------------------------ epilogue (as the bf16 swap tiles)
         const GemmProblem& pr = P.prob[0];
         const int ew = warp - 2;
-        const int q = warp & 3;                // TMEM lane quarter this warp may access
-        const int c0 = (ew >> 2) * CW;         // accumulator columns (tokens) this warp owns
+        const int q = warp & 3;
+        const int c0 = (ew >> 2) * CW;
         const int lane_row = q * 32 + lane;
         int buf = 0;
         uint32_t bphase = 0;
@@ -310,17 +326,17 @@ __global__ void __launch_bounds__(Fp4Shape<BN, STAGES, KB, G>::kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, S::kTmemCols);
+        tmem_dealloc(tmem_base, 512);
     }
 }
 
-template <int BN, int STAGES, int KB, int G>
-cudaError_t launch_nvfp4(const TcParams& P, int grid, cudaStream_t s) {
-    using F = Fp4Shape<BN, STAGES, KB, G>;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4<BN, STAGES, KB, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)F::kSmem);
+template <int BN, int STAGES, int KB, int G, int AS>
+cudaError_t launch_nvfp4_tm(const TcParams& P, int grid, cudaStream_t s) {
+    using F = Fp4TmShape<BN, STAGES, KB, G, AS>;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F::kSmem);
     if (e != cudaSuccess) return e;
-    k_gemm_nvfp4<BN, STAGES, KB, G><<<grid, F::kThreads, F::kSmem, s>>>(P);
+    k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS><<<grid, F::kThreads, F::kSmem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -335,11 +351,11 @@ cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmP
     fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
     const int grid = tc_num_sms();
     switch (bn) {
-#ifndef LMOE_FP4_DEC
-#define LMOE_FP4_DEC 4, 2, 4   // stages, k-blocks per stage, dequantisation groups
-#endif
-        case kDecodeTN: return launch_nvfp4<kDecodeTN, LMOE_FP4_DEC>(P, grid, s);
-        case 128: return launch_nvfp4<128, 3, 2, 2>(P, grid, s);
+        case kDecodeTN:
+            // four k-blocks per stage where K allows (a multiple of 256), else two
+            if ((probs[0].kdim[0] / kBK) % 4 == 0) return launch_nvfp4_tm<kDecodeTN, 5, 4, 2, 2>(P, grid, s);
+            return launch_nvfp4_tm<kDecodeTN, 8, 2, 2, 4>(P, grid, s);
+        case 128: return launch_nvfp4_tm<128, 5, 2, 1, 4>(P, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }
