@@ -191,3 +191,28 @@ def test_nvfp4_ultra_prefill_sampled():
     rng = np.random.default_rng(23)
     T = ULTRA_PREFILL.T
     _nvfp4_sampled(ULTRA_PREFILL, np.sort(np.concatenate([[T - 1], rng.choice(T - 1, 2, replace=False)])))
+
+
+def test_nvfp4_inside_the_pre_norm_residual_block():
+    # the block (y = x + layer(rmsnorm(x))) with NVFP4 experts
+    import torch
+    shape = RAGGED4
+    layer, dev, q = nvfp4_layer(shape)
+    rng = np.random.default_rng(31)
+    g = torch.from_numpy(rng.uniform(0.5, 1.5, shape.H).astype(np.float32)).to(torch.bfloat16).cuda()
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    y = layer.forward_block(dev["x"], g, 1e-5, idx=idx)
+    torch.cuda.synchronize()
+    host = synth.host_inputs(shape)
+    wts = oracle_experts(shape, host, q, range(shape.E), dict(host))
+    yref, iref, _ = oracle.forward_block(oracle.make_cfg(shape), host["x"], H.bf16_to_bits(g), 1e-5, wts)
+    assert np.array_equal(idx.cpu().numpy(), iref)
+    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref)
+    print("nvfp4 block max_abs=%.3g rel_fro=%.3g" % (ma, rf))
+
+
+def test_nvfp4_ultra_skew_sampled():
+    # hot experts with thousands of tokens each run the 128-token NVFP4 tiles
+    from synth import ULTRA_SKEW
+    rng = np.random.default_rng(24)
+    _nvfp4_sampled(ULTRA_SKEW, np.sort(rng.choice(ULTRA_SKEW.T, 3, replace=False)))
