@@ -81,6 +81,9 @@ typedef struct {
     lmoe_dtype x_dtype;      /* dtype of x                                       */
     lmoe_mode mode;          /* BF16 (tensor cores) or FP32 (validation)         */
     lmoe_expert_format expert_format;  /* BF16 (default) or NVFP4               */
+    int local_experts;       /* expert parallelism: experts whose up/down weights
+                                this handle holds (0 = all E)                     */
+    int expert_base;         /* first of them (global expert id)                  */
 } lmoe_config;
 /* Supported: E <= 1024, k <= min(64, Gk * E / G), E / G >= 2 when G > 1.
  * NVFP4 experts: mode LMOE_MODE_BF16, I and L multiples of 128. */
@@ -161,6 +164,45 @@ lmoe_status latentmoe_forward_block(lmoe_handle* h, const void* x, int T, const 
  * before latentmoe_create. */
 lmoe_status latentmoe_quantize_nvfp4(const void* w, long long n_mat, int R, int K, void* codes, void* sf, float* gs,
                                      void* stream);
+
+/* ---- Expert parallelism --------------------------------------------------
+ * The layer split into the three stages around the exchange of expert
+ * parallelism ("Nemotron-3-Labs-Ultra-Math-SFT" article: section 什么是 Latent
+ * 瓶颈, the experts exchange 2048-wide latent rows, a quarter of the hidden
+ * width, to cut the traffic of multi-GPU expert parallelism; deployment notes:
+ * the 512 experts sharded over the GPUs). The experts are partitioned
+ * over P ranks in contiguous blocks of E/P ids; each rank's handle holds the
+ * router, fc1/fc2 and the shared expert in full and the up/down weights of its
+ * own block only (local_experts = E/P, expert_base = rank * E/P). Per forward:
+ *   1 latentmoe_ep_front   routing, z = fc1(x), a_s, and the rows of z in
+ *                          expert order (send_rows [T*k, L] bf16) with their
+ *                          routing weights (send_w [T*k] fp32) and the
+ *                          per-expert counts [E]; rows for rank r are the
+ *                          rows of experts r*E/P .. (r+1)*E/P-1, contiguous.
+ *   (caller) exchange counts and rows all-to-all (rows of source s arrive in
+ *            expert order; recv_counts [n_src, local_experts] int32)
+ *   2 latentmoe_ep_experts the local experts on the received rows in their
+ *                          arrival order: recv_o = w * down(relu2(up(row)))
+ *                          [n_rows, L] fp32, same order (the weights are
+ *                          applied here, as in the single-GPU path)
+ *   (caller) return recv_o to the sources all-to-all (in the order they sent)
+ *   3 latentmoe_ep_back    combine the k returned rows of each token in
+ *                          ascending expert id, y = comb W_fc2^T + a_s W_sd^T
+ * Steps 1 and 3 use the same workspace (sized by latentmoe_workspace_size(T)),
+ * which carries the permutation and a_s between them; step 2 its own
+ * (latentmoe_ep_workspace_size). With P = 1 the three steps give the same y
+ * bit for bit as latentmoe_forward. All pointers are device memory. */
+lmoe_status latentmoe_ep_front(lmoe_handle* h, const void* x, int T, void* send_rows, float* send_w,
+                               int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream);
+/* recv_counts: device int32 [n_src * local_experts] (source-major); n_rows =
+ * their sum; n_src * local_experts <= 1024. */
+lmoe_status latentmoe_ep_workspace_size(const lmoe_handle* h, int n_rows, int n_src, size_t* bytes);
+lmoe_status latentmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const float* recv_w,
+                                 const int32_t* recv_counts, int n_src, int n_rows, float* recv_o, void* ws,
+                                 size_t ws_bytes, void* stream);
+/* send_o: [T*k, L] fp32, row i = the result for send_rows row i. */
+lmoe_status latentmoe_ep_back(lmoe_handle* h, const float* send_o, int T, float* y, void* ws, size_t ws_bytes,
+                              void* stream);
 
 /* Releases the handle (host memory only). */
 void latentmoe_destroy(lmoe_handle* h);

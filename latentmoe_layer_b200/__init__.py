@@ -28,7 +28,8 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
            "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias", "latentmoe_forward_block",
-           "latentmoe_quantize_nvfp4"]
+           "latentmoe_quantize_nvfp4", "latentmoe_ep_front", "latentmoe_ep_workspace_size", "latentmoe_ep_experts",
+           "latentmoe_ep_back"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -36,7 +37,7 @@ class lmoe_config(ctypes.Structure):
                 ("top_k", ctypes.c_int), ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int),
                 ("expert_inter", ctypes.c_int), ("shared_inter", ctypes.c_int), ("max_tokens", ctypes.c_int),
                 ("routed_scaling_factor", ctypes.c_float), ("x_dtype", ctypes.c_int), ("mode", ctypes.c_int),
-                ("expert_format", ctypes.c_int)]
+                ("expert_format", ctypes.c_int), ("local_experts", ctypes.c_int), ("expert_base", ctypes.c_int)]
 
 
 class lmoe_weights(ctypes.Structure):
@@ -86,10 +87,15 @@ def load():
     lib.latentmoe_update_bias.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp]
     lib.latentmoe_forward_block.argtypes = [vp, vp, i32, vp, ctypes.c_float, vp, vp, sz, vp, vp, vp, vp]
     lib.latentmoe_quantize_nvfp4.argtypes = [vp, ctypes.c_longlong, i32, i32, vp, vp, vp, vp]
+    lib.latentmoe_ep_front.argtypes = [vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.latentmoe_ep_workspace_size.argtypes = [vp, i32, i32, ctypes.POINTER(sz)]
+    lib.latentmoe_ep_experts.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+    lib.latentmoe_ep_back.argtypes = [vp, vp, i32, vp, vp, sz, vp]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
               "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias",
-              "latentmoe_forward_block", "latentmoe_quantize_nvfp4"):
+              "latentmoe_forward_block", "latentmoe_quantize_nvfp4", "latentmoe_ep_front",
+              "latentmoe_ep_workspace_size", "latentmoe_ep_experts", "latentmoe_ep_back"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -192,13 +198,14 @@ class LatentMoE:
     """
 
     def __init__(self, shape, weights: dict, max_tokens: int, x_f32: bool = False, mode: int = LMOE_MODE_BF16,
-                 expert_format: int = LMOE_EXPERTS_BF16):
+                 expert_format: int = LMOE_EXPERTS_BF16, local_experts: int = 0, expert_base: int = 0):
         import torch
         self.torch = torch
         self.shape = shape
         self.weights = weights
         cfg = lmoe_config(shape.H, shape.L, shape.E, shape.k, shape.G, shape.Gk, shape.I, shape.Is, max_tokens,
-                          float(shape.s), LMOE_FP32 if x_f32 else LMOE_BF16, mode, expert_format)
+                          float(shape.s), LMOE_FP32 if x_f32 else LMOE_BF16, mode, expert_format, local_experts,
+                          expert_base)
         w = lmoe_weights(*[_p(weights.get(n)) for n in ("router_w", "e_bias", "fc1_w", "fc2_w", "up_w", "down_w",
                                                          "shared_up_w", "shared_down_w", "up_sf", "down_sf",
                                                          "up_gs", "down_gs")])
@@ -211,6 +218,7 @@ class LatentMoE:
         self.mode = mode
         self._ws = None
         self._ws_T = -1
+        self._ep_ws = None
 
     def workspace(self, T: int):
         s, n = latentmoe_workspace_size(self.h, T)
@@ -251,6 +259,40 @@ class LatentMoE:
         if s != LMOE_OK:
             raise LmoeError(s, "latentmoe_forward_block")
         return y
+
+    # ---- expert parallelism (the three stages around the all-to-all exchange)
+    def ep_front(self, x, send_rows, send_w, counts):
+        """Routing, fc1 + shared up, and the rows of z in expert order (send_rows
+        [T*k, L] bf16, send_w [T*k] fp32, counts [E] int32). Keeps the workspace
+        state that ep_back needs."""
+        T = x.shape[0]
+        ws, n = self.workspace(T)
+        s = load().latentmoe_ep_front(self.h, _p(x), T, _p(send_rows), _p(send_w), _p(counts), _p(ws), ws.numel(),
+                                      self._stream())
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_ep_front")
+
+    def ep_experts(self, recv_rows, recv_w, recv_counts, n_src, recv_o):
+        """This handle's experts on received rows (source-major, expert order within a source)."""
+        n_rows = recv_rows.shape[0]
+        nbytes = ctypes.c_size_t()
+        s = load().latentmoe_ep_workspace_size(self.h, n_rows, n_src, ctypes.byref(nbytes))
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_ep_workspace_size")
+        if self._ep_ws is None or self._ep_ws.numel() < nbytes.value:
+            self._ep_ws = self.torch.empty(max(nbytes.value, 256), dtype=self.torch.uint8, device="cuda")
+        s = load().latentmoe_ep_experts(self.h, _p(recv_rows), _p(recv_w), _p(recv_counts), n_src, n_rows,
+                                        _p(recv_o), _p(self._ep_ws), self._ep_ws.numel(), self._stream())
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_ep_experts")
+
+    def ep_back(self, send_o, y):
+        """Combine the returned rows (send order) and the output GEMM into y [T, H] fp32."""
+        T = y.shape[0]
+        ws, n = self.workspace(T)
+        s = load().latentmoe_ep_back(self.h, _p(send_o), T, _p(y), _p(ws), ws.numel(), self._stream())
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_ep_back")
 
     def route(self, x, idx=None, w=None, counts=None):
         torch = self.torch

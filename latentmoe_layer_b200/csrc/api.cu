@@ -132,6 +132,9 @@ lmoe_status check_config(const lmoe_config* c) {
     if (c->expert_format == LMOE_EXPERTS_NVFP4 &&
         (c->mode != LMOE_MODE_BF16 || c->expert_inter % 128 || c->latent % 128))
         return LMOE_ERR_UNSUPPORTED;  // weight tiles of 128 rows; tensor-core path only
+    if (c->local_experts < 0 || c->expert_base < 0 || c->local_experts > c->num_experts ||
+        (long long)c->expert_base + (c->local_experts ? c->local_experts : c->num_experts) > c->num_experts)
+        return LMOE_ERR_INVALID_ARG;
     if (c->num_experts > kMaxE || c->n_group > kMaxG || c->top_k > kMaxK) return LMOE_ERR_UNSUPPORTED;
     if (c->n_group > 1 && c->num_experts / c->n_group < 2) return LMOE_ERR_UNSUPPORTED;
     if (c->hidden > 16384) return LMOE_ERR_UNSUPPORTED;  // fp64 router stages one x row in shared memory
@@ -357,26 +360,19 @@ __global__ void k_publish_error(const int* derr, int* herr) {
 
 // The layer on x (launches 1-10 of the file comment). With `resid` (bf16
 // [T, H]) the output GEMM adds it: y = resid + layer(x).
-lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y, void* ws, void* stream,
-                         int32_t* topk_idx, float* topk_w, int32_t* expert_counts, const uint16_t* resid,
-                         const uint16_t* norm_src, const uint16_t* norm_w, double norm_eps) {
-    lmoe_status s;
-    const lmoe_config& cf = h->cfg;
-    Ctx c = make_ctx(h, p, ws, stream);
-    char* ws_c = c.ws;
-    h->launches = 0;
-    mark(c, 0);
-    if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
-                                                reinterpret_cast<uint16_t*>(const_cast<void*>(x)), c.s));
-    s = do_route(c, x, topk_idx, topk_w, expert_counts);
-    if (s != LMOE_OK) return s;
-    mark(c, 1);
-    const int gemm_kernels = c.simt ? 2 : 1;  // SIMT launches one kernel per problem
+int experts_held(const lmoe_config& c) { return c.local_experts > 0 ? c.local_experts : c.num_experts; }
 
+// Steps 5-6: z = x W_fc1^T and a_s = relu2(x W_su^T) (one launch), then the
+// rows of z in expert order (the permutation of do_route) into zdst.
+lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const Plan& p = *c.p;
+    char* ws_c = c.ws;
     const bool bf16 = cf.mode == LMOE_MODE_BF16;
     const int act = bf16 ? 2 : 4;
-    const int H = cf.hidden, L = cf.latent, I = cf.expert_inter, Is = cf.shared_inter, E = cf.num_experts;
-    const long long A = p.A;
+    const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter, E = cf.num_experts;
+    const int gemm_kernels = c.simt ? 2 : 1;  // SIMT launches one kernel per problem
     // GEMM operand x: bf16 x as given, fp32 x rounded to bf16 (bf16 mode) or fp32 x (validation mode).
     const void* xa = x;
     bool xa_f32 = cf.x_dtype == LMOE_FP32;
@@ -386,13 +382,9 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         xa = ws_c + p.xbf;
         xa_f32 = false;
     }
-    const int epi_act = bf16 ? EPI_BF16 : EPI_F32;
-    const int epi_relu2 = bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32;
-
-    // 5: z = x W_fc1^T, a_s = relu2(x W_su^T)
     {
-        GemmProblem pr[2] = {make_problem(0, p.T, L, epi_act, ws_c + p.z, L),
-                             make_problem(0, p.T, Is, epi_relu2, ws_c + p.as, Is)};
+        GemmProblem pr[2] = {make_problem(0, p.T, L, bf16 ? EPI_BF16 : EPI_F32, ws_c + p.z, L),
+                             make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is)};
         pr[0].kdim[0] = H;
         pr[1].kdim[0] = H;
         pr[0].a_ptr[0] = xa;
@@ -404,20 +396,31 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
     }
     mark(c, 2);
-    // 6: expert-ordered copy of z
-    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, ws_c + p.zperm, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
+    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
                                       reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
     mark(c, 3);
+    return LMOE_OK;
+}
+
+// Steps 7-8 on n rows grouped as c.r describes: a = relu2(rows W_up[e]^T) into
+// a_buf, o = w * (a W_down[e]^T) (NVFP4: the matrix scales before relu2 and w).
+// Group g takes expert g % expert_mod's weights when expert_mod is non-zero.
+lmoe_status stage_experts(Ctx& c, const void* rows, long long n, const float* row_w, void* a_buf, float* o,
+                          int expert_mod) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const bool bf16 = cf.mode == LMOE_MODE_BF16;
     const bool fp4 = cf.expert_format == LMOE_EXPERTS_NVFP4;
-    // 7: a = relu2(z_e W_up[e]^T)   (NVFP4: relu2(g_e * (z_e (codes * scales)^T)))
+    const int L = cf.latent, I = cf.expert_inter, Ew = experts_held(cf);
     {
-        GemmProblem pr = make_problem(1, 0, I, epi_relu2, ws_c + p.aperm, I);
+        GemmProblem pr = make_problem(1, 0, I, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, a_buf, I);
         pr.kdim[0] = L;
         pr.b_rows_per_expert = I;
-        pr.a_ptr[0] = ws_c + p.zperm;
+        pr.expert_mod = expert_mod;
+        pr.a_ptr[0] = rows;
         pr.b_ptr[0] = h->w.up_w;
-        Operand a[1][2] = {{{ws_c + p.zperm, A}, {nullptr, 0}}};
-        Operand b[1][2] = {{{h->w.up_w, (long long)E * I}, {nullptr, 0}}};
+        Operand a[1][2] = {{{rows, n}, {nullptr, 0}}};
+        Operand b[1][2] = {{{h->w.up_w, (long long)Ew * I}, {nullptr, 0}}};
         if (fp4) {
             pr.wq_codes = static_cast<const uint8_t*>(h->w.up_w);
             pr.wq_sf = static_cast<const uint8_t*>(h->w.up_sf);
@@ -428,16 +431,16 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         }
     }
     mark(c, 4);
-    // 8: o = w * (a_e W_down[e]^T)
     {
-        GemmProblem pr = make_problem(1, 0, L, EPI_SCALE_F32, ws_c + p.o, L);
+        GemmProblem pr = make_problem(1, 0, L, EPI_SCALE_F32, o, L);
         pr.kdim[0] = I;
         pr.b_rows_per_expert = L;
-        pr.row_scale = reinterpret_cast<const float*>(ws_c + p.wperm);
-        pr.a_ptr[0] = ws_c + p.aperm;
+        pr.expert_mod = expert_mod;
+        pr.row_scale = row_w;
+        pr.a_ptr[0] = a_buf;
         pr.b_ptr[0] = h->w.down_w;
-        Operand a[1][2] = {{{ws_c + p.aperm, A}, {nullptr, 0}}};
-        Operand b[1][2] = {{{h->w.down_w, (long long)E * L}, {nullptr, 0}}};
+        Operand a[1][2] = {{{a_buf, n}, {nullptr, 0}}};
+        Operand b[1][2] = {{{h->w.down_w, (long long)Ew * L}, {nullptr, 0}}};
         if (fp4) {
             pr.wq_codes = static_cast<const uint8_t*>(h->w.down_w);
             pr.wq_sf = static_cast<const uint8_t*>(h->w.down_sf);
@@ -448,11 +451,22 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         }
     }
     mark(c, 5);
-    // 9: comb
-    LMOE_LAUNCH(1, launch_combine(reinterpret_cast<const float*>(ws_c + p.o), reinterpret_cast<const int*>(ws_c + p.slot),
-                                  ws_c + p.comb, p.T, cf.top_k, L, bf16, c.s));
+    return LMOE_OK;
+}
+
+// Steps 9-10: comb[t] = bf16(sum of the token's k rows of o, ascending expert
+// id) via the slot map of do_route, then y = comb W_fc2^T + a_s W_sd^T
+// (+ resid), one K-concatenated GEMM.
+lmoe_status stage_back(Ctx& c, const float* o, float* y, const uint16_t* resid) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const Plan& p = *c.p;
+    char* ws_c = c.ws;
+    const bool bf16 = cf.mode == LMOE_MODE_BF16;
+    const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter;
+    LMOE_LAUNCH(1, launch_combine(o, reinterpret_cast<const int*>(ws_c + p.slot), ws_c + p.comb, p.T, cf.top_k, L,
+                                  bf16, c.s));
     mark(c, 6);
-    // 10: y = comb W_fc2^T + a_s W_sd^T
     {
         GemmProblem pr = make_problem(0, p.T, H, EPI_F32, y, H);
         pr.nseg = 2;
@@ -468,9 +482,63 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
         LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
     }
     mark(c, 7);
+    return LMOE_OK;
+}
+
+lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y, void* ws, void* stream,
+                         int32_t* topk_idx, float* topk_w, int32_t* expert_counts, const uint16_t* resid,
+                         const uint16_t* norm_src, const uint16_t* norm_w, double norm_eps) {
+    lmoe_status s;
+    const lmoe_config& cf = h->cfg;
+    Ctx c = make_ctx(h, p, ws, stream);
+    char* ws_c = c.ws;
+    h->launches = 0;
+    mark(c, 0);
+    if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
+                                                reinterpret_cast<uint16_t*>(const_cast<void*>(x)), c.s));
+    s = do_route(c, x, topk_idx, topk_w, expert_counts);
+    if (s != LMOE_OK) return s;
+    mark(c, 1);
+    s = stage_front(c, x, ws_c + p.zperm);
+    if (s != LMOE_OK) return s;
+    s = stage_experts(c, ws_c + p.zperm, p.A, reinterpret_cast<const float*>(ws_c + p.wperm), ws_c + p.aperm,
+                      reinterpret_cast<float*>(ws_c + p.o), 0);
+    if (s != LMOE_OK) return s;
+    s = stage_back(c, reinterpret_cast<const float*>(ws_c + p.o), y, resid);
+    if (s != LMOE_OK) return s;
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
     h->launches += 1;
     return cuda_status(cudaGetLastError());
+}
+
+// Workspace of latentmoe_ep_experts: the scan of the received blocks and the
+// expert activations of the received rows.
+struct EpPlan {
+    size_t total, stats, bcounts, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64, rec128, rec256, a;
+};
+
+void ep_plan_of(const lmoe_config& c, int n_rows, int nb, EpPlan& p) {
+    const size_t n = n_rows;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += al256(bytes);
+        return o;
+    };
+    p.stats = take(sizeof(WsStats));
+    p.bcounts = take((size_t)nb * 4);
+    p.counts = take((size_t)nb * 4);
+    p.offsets = take((size_t)(nb + 1) * 4);
+    p.pfx128 = take((size_t)(nb + 1) * 4);
+    p.pfx64 = take((size_t)(nb + 1) * 4);
+    p.pfxdec = take((size_t)(nb + 1) * 4);
+    p.pfx256 = take((size_t)(nb + 1) * 4);
+    p.rec32 = take((n / 32 + nb) * 16);
+    p.rec64 = take((n / 64 + nb) * 16);
+    p.rec128 = take((n / 128 + nb) * 16);
+    p.rec256 = take((n / 256 + nb) * 16);
+    p.a = take(n * c.expert_inter * (c.mode == LMOE_MODE_BF16 ? 2 : 4));
+    p.total = off;
 }
 
 lmoe_status check_outputs(float* y, int32_t* topk_idx, float* topk_w, int32_t* expert_counts) {
@@ -490,6 +558,7 @@ lmoe_status latentmoe_forward(lmoe_handle* h, const void* x, int T, float* y, vo
     Plan p;
     lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
     if (s != LMOE_OK || T == 0) return s;
+    if (experts_held(h->cfg) != h->cfg.num_experts) return LMOE_ERR_UNSUPPORTED;  // a shard: use the ep_ calls
     s = check_outputs(y, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
     s = take_device_error(h);
@@ -503,7 +572,7 @@ lmoe_status latentmoe_forward_block(lmoe_handle* h, const void* x, int T, const 
     Plan p;
     lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
     if (s != LMOE_OK || T == 0) return s;
-    if (h->cfg.x_dtype != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
+    if (h->cfg.x_dtype != LMOE_BF16 || experts_held(h->cfg) != h->cfg.num_experts) return LMOE_ERR_UNSUPPORTED;
     if (!norm_w || !aligned(norm_w, 16) || !(norm_eps >= 0.f) || isinf(norm_eps)) return LMOE_ERR_INVALID_ARG;
     s = check_outputs(y, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
@@ -630,6 +699,116 @@ lmoe_status latentmoe_update_bias(lmoe_handle* h, const int32_t* expert_counts, 
         return LMOE_ERR_INVALID_ARG;
     return cuda_status(launch_update_bias(expert_counts, bias_in, h->cfg.num_experts, (double)eta, bias_out, maxvio_out,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+lmoe_status latentmoe_ep_front(lmoe_handle* h, const void* x, int T, void* send_rows, float* send_w,
+                               int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    lmoe_status s = validate_call(h, x, T, ws, ws_bytes, p);
+    if (s != LMOE_OK || T == 0) return s;
+    if (!send_rows || !aligned(send_rows, 16) || !send_w || !aligned(send_w, 4) || !expert_counts ||
+        !aligned(expert_counts, 4))
+        return LMOE_ERR_INVALID_ARG;
+    s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    Ctx c = make_ctx(h, p, ws, stream);
+    h->launches = 0;
+    mark(c, 0);
+    s = do_route(c, x, nullptr, nullptr, expert_counts);
+    if (s != LMOE_OK) return s;
+    mark(c, 1);
+    s = stage_front(c, x, send_rows);
+    if (s != LMOE_OK) return s;
+    LMOE_TRY(cudaMemcpyAsync(send_w, c.ws + p.wperm, (size_t)p.A * 4, cudaMemcpyDeviceToDevice, c.s));
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+lmoe_status latentmoe_ep_workspace_size(const lmoe_handle* h, int n_rows, int n_src, size_t* bytes) {
+    if (!h || !bytes || n_rows < 0 || n_src < 1) return LMOE_ERR_INVALID_ARG;
+    const int nb = n_src * experts_held(h->cfg);
+    if (nb > kMaxE) return LMOE_ERR_UNSUPPORTED;
+    EpPlan p;
+    ep_plan_of(h->cfg, n_rows, nb, p);
+    *bytes = p.total;
+    return LMOE_OK;
+}
+
+lmoe_status latentmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const float* recv_w,
+                                 const int32_t* recv_counts, int n_src, int n_rows, float* recv_o, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    if (!h || n_src < 1 || n_rows < 0 || !recv_counts || !aligned(recv_counts, 4)) return LMOE_ERR_INVALID_ARG;
+    const lmoe_config& cf = h->cfg;
+    const int El = experts_held(cf), nb = n_src * El;
+    if (nb > kMaxE || (long long)n_rows > (long long)cf.max_tokens * cf.top_k * n_src) return LMOE_ERR_UNSUPPORTED;
+    if (n_rows == 0) return LMOE_OK;
+    if (!recv_rows || !aligned(recv_rows, 16) || !recv_w || !aligned(recv_w, 4) || !recv_o || !aligned(recv_o, 16))
+        return LMOE_ERR_INVALID_ARG;
+    EpPlan q;
+    ep_plan_of(cf, n_rows, nb, q);
+    if (!ws || !aligned(ws, 256) || ws_bytes < q.total) return LMOE_ERR_WORKSPACE;
+    lmoe_status s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    // a plan carrying only what the GEMM launchers read (row count of the grouped problems)
+    Plan p;
+    memset(&p, 0, sizeof(p));
+    p.T = n_rows;
+    p.A = n_rows;
+    Ctx c;
+    c.h = h;
+    c.p = &p;
+    c.ws = static_cast<char*>(ws);
+    c.s = static_cast<cudaStream_t>(stream);
+    c.r.offsets = reinterpret_cast<const int*>(c.ws + q.offsets);
+    c.r.pfx128 = reinterpret_cast<const int*>(c.ws + q.pfx128);
+    c.r.pfx64 = reinterpret_cast<const int*>(c.ws + q.pfx64);
+    c.r.pfxdec = reinterpret_cast<const int*>(c.ws + q.pfxdec);
+    c.r.pfx256 = reinterpret_cast<const int*>(c.ws + q.pfx256);
+    c.r.rec32 = reinterpret_cast<const int4*>(c.ws + q.rec32);
+    c.r.rec64 = reinterpret_cast<const int4*>(c.ws + q.rec64);
+    c.r.rec128 = reinterpret_cast<const int4*>(c.ws + q.rec128);
+    c.r.rec256 = reinterpret_cast<const int4*>(c.ws + q.rec256);
+    c.r.E = nb;
+    c.err = &reinterpret_cast<WsStats*>(c.ws + q.stats)->device_error;
+    c.simt = h->gemm_path == 3 || cf.mode == LMOE_MODE_FP32;
+    if (h->gemm_path == 1 || h->gemm_path == 4) c.decode = false;
+    else if (h->gemm_path == 2) c.decode = true;
+    else c.decode = (long long)n_rows <= 64LL * El * n_src;  // <= 64 rows per block on average, as the forward
+    h->launches = 0;
+    LMOE_TRY(cudaMemsetAsync(c.ws + q.stats, 0, sizeof(WsStats), c.s));
+    LMOE_TRY(cudaMemcpyAsync(c.ws + q.bcounts, recv_counts, (size_t)nb * 4, cudaMemcpyDeviceToDevice, c.s));
+    LMOE_LAUNCH(2, launch_group_scan(reinterpret_cast<int*>(c.ws + q.bcounts), nb, n_rows,
+                                     reinterpret_cast<int*>(c.ws + q.counts), reinterpret_cast<int*>(c.ws + q.offsets),
+                                     reinterpret_cast<int*>(c.ws + q.pfx128), reinterpret_cast<int*>(c.ws + q.pfx64),
+                                     reinterpret_cast<int*>(c.ws + q.pfxdec), reinterpret_cast<int*>(c.ws + q.pfx256),
+                                     reinterpret_cast<int4*>(c.ws + q.rec32), reinterpret_cast<int4*>(c.ws + q.rec64),
+                                     reinterpret_cast<int4*>(c.ws + q.rec128), reinterpret_cast<int4*>(c.ws + q.rec256),
+                                     reinterpret_cast<WsStats*>(c.ws + q.stats), c.s));
+    s = stage_experts(c, recv_rows, n_rows, recv_w, c.ws + q.a, recv_o, El);
+    if (s != LMOE_OK) return s;
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+lmoe_status latentmoe_ep_back(lmoe_handle* h, const float* send_o, int T, float* y, void* ws, size_t ws_bytes,
+                              void* stream) {
+    if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    if (T == 0) return LMOE_OK;
+    Plan p;
+    plan_of(h->cfg, T, p);
+    if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return LMOE_ERR_WORKSPACE;
+    if (!send_o || !aligned(send_o, 16) || !y || !aligned(y, 16)) return LMOE_ERR_INVALID_ARG;
+    lmoe_status s = take_device_error(h);
+    if (s != LMOE_OK) return s;
+    Ctx c = make_ctx(h, p, ws, stream);
+    h->launches = 0;
+    s = stage_back(c, send_o, y, nullptr);
+    if (s != LMOE_OK) return s;
+    k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
 }
 
 lmoe_status latentmoe_quantize_nvfp4(const void* w, long long n_mat, int R, int K, void* codes, void* sf, float* gs,

@@ -116,7 +116,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         const int nct = n_col_tiles(pr, S::kOutCols);
         const int mt = t / nct, ct = t % nct;
         const int4 rc = __ldg(grouped_records<S::kActRows>(P.r) + mt);
-        const int e = rc.x;
+        const int e = pr.expert_mod ? rc.x % pr.expert_mod : rc.x;
         ti.p = 0;
         ti.row0 = rc.y;
         ti.rows = rc.z;

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const GemmProblem pr, const D
         }
         row0 = r.offsets[lo] + (mt - r.pfx64[lo]) * TM;
         rows = min(TM, r.offsets[lo + 1] - row0);
-        wrow0 = lo * pr.b_rows_per_expert + col0;
+        wrow0 = (pr.expert_mod ? lo % pr.expert_mod : lo) * pr.b_rows_per_expert + col0;
     } else {
         row0 = blockIdx.x * TM;
         rows = min(TM, pr.m_rows - row0);

@@ -299,8 +299,8 @@ __device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32
         const int4 rc = __ldg(P.r.rec256 + mt);
         prow0 = rc.y;
         prows = rc.z;
-        wbase = rc.x * pr.b_rows_per_expert;
-        e = rc.x;
+        e = pr.expert_mod ? rc.x % pr.expert_mod : rc.x;
+        wbase = e * pr.b_rows_per_expert;
     } else {
         if (P.nprob > 1 && t >= P.dense_tiles[0]) {
             t -= P.dense_tiles[0];

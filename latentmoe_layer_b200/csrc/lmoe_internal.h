@@ -61,6 +61,10 @@ struct GemmProblem {
     const uint8_t* wq_codes;  // tile t at wq_codes + 4096 t
     const uint8_t* wq_sf;     // tile t at wq_sf + 512 t
     const float* wscale;      // [E] matrix scale per expert
+    // Grouped problems: when non-zero, group g uses the weights of expert
+    // g % expert_mod (expert parallelism: groups are (source rank, local expert)
+    // blocks of received rows in arrival order).
+    int expert_mod;
 };
 
 struct DeviceRouting {
@@ -98,6 +102,9 @@ cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Pl
                                    cudaStream_t s);
 cudaError_t launch_router_select64(const lmoe_handle* h, const Plan& p, char* ws, bool all, cudaStream_t s);
 cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_t* counts_out, cudaStream_t s);
+cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts, int* offsets, int* pfx128, int* pfx64,
+                              int* pfxdec, int* pfx256, int4* rec32, int4* rec64, int4* rec128, int4* rec256,
+                              WsStats* st, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* offsets_E,
                                int row_bytes, cudaStream_t s);
 cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,

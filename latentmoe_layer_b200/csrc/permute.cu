@@ -370,6 +370,30 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
     return cudaGetLastError();
 }
 
+// Rows received for expert parallelism: blockcounts holds the count of each
+// (source rank, local expert) block (one "block row" of the scan); the scan
+// gives its offsets, tile prefixes and tile records. If the counts do not add
+// up to n_rows the tile prefixes are zeroed (no GEMM tile runs) and
+// LMOE_ERR_INVALID_ARG is recorded.
+__global__ void k_check_rows(const int* __restrict__ offsets, int nb, int n_rows, int* pfx128, int* pfx64, int* pfxdec,
+                             int* pfx256, WsStats* st) {
+    if (threadIdx.x == 0 && offsets[nb] != n_rows) {
+        pfx128[nb] = pfx64[nb] = pfxdec[nb] = pfx256[nb] = 0;
+        atomicCAS(&st->device_error, 0, (int)LMOE_ERR_INVALID_ARG);
+    }
+}
+
+cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts, int* offsets, int* pfx128, int* pfx64,
+                              int* pfxdec, int* pfx256, int4* rec32, int4* rec64, int4* rec128, int4* rec256,
+                              WsStats* st, cudaStream_t s) {
+    k_scan<<<1, 1024, 0, s>>>(blockcounts, 1, nb, counts, nullptr, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64,
+                              rec128, rec256, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_check_rows<<<1, 32, 0, s>>>(offsets, nb, n_rows, pfx128, pfx64, pfxdec, pfx256, st);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* total,
                                int row_bytes, cudaStream_t s) {
     const int vpr = row_bytes / 16;

@@ -85,6 +85,25 @@ def test_nvfp4_configs_rejected_before_any_cuda_call(lib, kw, status):
     assert s == status and not h.value
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(local_experts=-1), lm.LMOE_ERR_INVALID_ARG),
+    (dict(local_experts=17), lm.LMOE_ERR_INVALID_ARG),             # more than E
+    (dict(local_experts=8, expert_base=9), lm.LMOE_ERR_INVALID_ARG),  # block past E
+    (dict(expert_base=-8), lm.LMOE_ERR_INVALID_ARG),
+])
+def test_expert_shard_configs_rejected_before_any_cuda_call(lib, kw, status):
+    s, h = lm.latentmoe_create(good_cfg(**kw), fake_weights())
+    assert s == status and not h.value
+
+
+def test_expert_parallel_entry_points_reject_null_handles(lib):
+    n = ctypes.c_size_t()
+    assert lib.latentmoe_ep_workspace_size(None, 4, 1, ctypes.byref(n)) == lm.LMOE_ERR_INVALID_ARG
+    assert lib.latentmoe_ep_front(None, None, 1, None, None, None, None, 0, None) == lm.LMOE_ERR_INVALID_ARG
+    assert lib.latentmoe_ep_experts(None, None, None, None, 1, 1, None, None, 0, None) == lm.LMOE_ERR_INVALID_ARG
+    assert lib.latentmoe_ep_back(None, None, 1, None, None, 0, None) == lm.LMOE_ERR_INVALID_ARG
+
+
 def test_nvfp4_weights_need_scales(lib):
     cfg = good_cfg(expert_format=lm.LMOE_EXPERTS_NVFP4, latent=128)
     for bad in (0, 0x10008):
