@@ -340,6 +340,35 @@ def cpu_baseline(shape, dev, target_s=15.0):
                       (done, shape.T), "seconds": round(t2 - t0, 2)}, wts
 
 
+def cpu_baseline_one_core(shape, wts, dev, target_s=8.0):
+    """The same oracle on one host core (its OpenMP runtime limited to one
+    thread for this measurement, then restored), over a smaller token sample."""
+    import ctypes
+    import numpy as np
+    import oracle
+    import torch
+    gomp = ctypes.CDLL("libgomp.so.1")
+    gomp.omp_get_max_threads.restype = ctypes.c_int
+    before = gomp.omp_get_max_threads()
+    xs = dev["x"].cpu().numpy() if shape.x_f32 else dev["x"].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    cfg = oracle.make_cfg(shape)
+    gomp.omp_set_num_threads(1)
+    try:
+        t0 = time.time()
+        oracle.forward(cfg, xs[:1], wts)
+        t1 = time.time()
+        more = int(min(shape.T - 1, max(0.0, target_s - (t1 - t0)) / max(t1 - t0, 1e-9)))
+        if more > 0:
+            oracle.forward(cfg, xs[1:1 + more], wts)
+        t2 = time.time()
+    finally:
+        gomp.omp_set_num_threads(before)
+    done = 1 + max(more, 0)
+    return {"value": round(done / (t2 - t0), 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d of %d tokens of the workload, full layer per token (fp64, one thread)" %
+                      (done, shape.T), "seconds": round(t2 - t0, 2)}
+
+
 def run_ours(args):
     import torch
     import synth
@@ -381,8 +410,9 @@ def run_ours(args):
     }
     layer, dev = res["layer"], res["dev"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not nv:
-        cb, _ = cpu_baseline(shape, dev)
+        cb, wts = cpu_baseline(shape, dev)
         line["cpu_baseline"] = cb
+        line["cpu_baseline_1core"] = cpu_baseline_one_core(shape, wts, dev)
     layer.close()
     del res, layer, dev
     torch.cuda.empty_cache()
