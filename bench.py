@@ -231,6 +231,13 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
     stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, name in enumerate(STAGES)}
     st = layer.stats()
+    # expert loads of this batch (one more, untimed forward that also writes the counts)
+    counts = torch.empty((shape.E,), dtype=torch.int32, device="cuda")
+    layer.forward(x, y, counts=counts)
+    cnt = counts.cpu().tolist()
+    loads = {"load_imbalance": round(max(cnt) / (shape.T * shape.k / shape.E), 3)}
+    if shape.skew_hot:
+        loads["hot_share"] = round(sum(cnt[:shape.skew_hot]) / float(shape.T * shape.k), 4)
 
     # End to end through the public call with host buffers: every step copies its
     # x from pinned host memory to the device, runs the layer and copies y back.
@@ -279,7 +286,8 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
         dist.barrier()
     e_ms = max_over_ranks(e2e_run(e_steps), dist, "cuda")
     res = {
-        "ms": ms, "stage_ms": stage_ms, "stats": st, "clocks": clk, "e2e_ms": e_ms, "e2e_steps": e_steps,
+        "ms": ms, "stage_ms": stage_ms, "stats": st, "loads": loads, "clocks": clk, "e2e_ms": e_ms,
+        "e2e_steps": e_steps,
         "h2d": x.numel() * x.element_size(), "d2h": y.numel() * 4, "layer": layer, "dev": dev,
     }
     return res
@@ -331,7 +339,7 @@ def layer_summary(shape, res, peaks, peak_src, steps, nvfp4=False):
         "layer_frac_of_hbm": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "stage_ms": {k: round(v, 4) for k, v in res["stage_ms"].items()},
         "distinct_experts": st.distinct_experts, "max_expert_tokens": st.max_expert_tokens,
-        "flagged_tokens": st.flagged_tokens,
+        "flagged_tokens": st.flagged_tokens, **res["loads"],
     }
 
 
