@@ -199,14 +199,27 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
     }
 }
 
-// dst[r, :] = src[perm[r], :] for r < offsets_E[0] (row_bytes multiple of 16).
-__global__ void k_gather(const uint4* __restrict__ src, uint4* __restrict__ dst, const int* __restrict__ perm,
-                         const int* __restrict__ total, int vec_per_row) {
+// dst[r, :] = src[perm[r], :] for r < *total (row_bytes multiple of 16). One
+// warp per row: the source row index is read once, and each lane keeps up to
+// eight 16-byte loads in flight before its stores.
+__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                const int* __restrict__ perm, const int* __restrict__ total,
+                                                int vec_per_row) {
     const int rows = *total;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)rows * vec_per_row;
-         i += (long long)gridDim.x * blockDim.x) {
-        const long long r = i / vec_per_row, c = i % vec_per_row;
-        dst[i] = src[(long long)perm[r] * vec_per_row + c];
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+        const uint4* s = src + (long long)__ldg(perm + r) * vec_per_row;
+        uint4* d = dst + (long long)r * vec_per_row;
+        int c = lane;
+        for (; c + 7 * 32 < vec_per_row; c += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = ld_global_nc_v4(s + c + 32 * j);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_global_v4(d + c + 32 * j, v[j]);
+        }
+        for (; c < vec_per_row; c += 32) st_global_v4(d + c, ld_global_nc_v4(s + c));
     }
 }
 
@@ -397,7 +410,7 @@ cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts,
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* total,
                                int row_bytes, cudaStream_t s) {
     const int vpr = row_bytes / 16;
-    int grid = grid_cap((long long)rows_total_max * vpr, 256, 148 * 16);
+    int grid = grid_cap((long long)rows_total_max * 32, 256, 148 * 8);  // one warp per row
     k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, total, vpr);
     return cudaGetLastError();
 }
