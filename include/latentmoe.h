@@ -233,7 +233,16 @@ typedef enum {
                                     the dense GEMMs, and 3 is unsupported (LMOE_ERR_UNSUPPORTED). */
     LMOE_OPT_ROUTER_FP64_ALL = 1,/* 1: every token's logits recomputed in fp64 (validation)      */
     LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin for the fp64 re-check, in 1e-9 units        */
-    LMOE_OPT_SPIN_LIMIT = 3      /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */
+    LMOE_OPT_SPIN_LIMIT = 3,     /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */
+    LMOE_OPT_Z_RECHECK_DELTA = 4 /* margin of the exact re-rounding of z, in 1e-9 units (default
+                                    5000 = 5e-6; 0 disables). bf16 mode, tensor-core GEMMs: the
+                                    fc1 product is kept in fp32, rounded to bf16 nearest-even,
+                                    and every element whose fp32 value lies within the margin of
+                                    a bf16 rounding midpoint is recomputed as an fp64 sum of the
+                                    exact bf16 products and rounded again, so z is the exactly
+                                    rounded x W_fc1^T whenever the fp32 error is below the margin
+                                    (z is the rounding point that every routed expert of a token
+                                    reads). Valid range 0 .. 1e8. */
 } lmoe_option;
 lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long value);
 
@@ -245,6 +254,7 @@ typedef struct {
     int kernel_launches;    /* kernels the last route/forward call on the handle launched */
     int cuda_error;         /* cudaError_t of the last CUDA runtime call on the handle that
                                failed (a call that returned LMOE_ERR_CUDA), 0 if none     */
+    int z_rechecked;        /* z elements re-rounded exactly (LMOE_OPT_Z_RECHECK_DELTA)    */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */

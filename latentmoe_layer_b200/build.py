@@ -7,7 +7,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "liblatentmoe.so")
-SOURCES = ["api.cu", "router.cu", "permute.cu", "gemm_tc.cu", "gemm_nvfp4.cu", "gemm_simt.cu", "nvfp4.cu"]
+SOURCES = ["api.cu", "router.cu", "permute.cu", "gemm_tc.cu", "gemm_nvfp4.cu", "gemm_simt.cu", "nvfp4.cu", "zcheck.cu"]
 HEADERS = ["lmoe_internal.h", "handle.h", "ptx.cuh", "gemm_common.cuh"]
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-Xcompiler", "-fPIC",
          "-shared", "--expt-relaxed-constexpr", "-Xptxas", "-v"]

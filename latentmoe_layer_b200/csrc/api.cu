@@ -17,6 +17,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <algorithm>
 #include <stdint.h>
 #include <string.h>
 
@@ -373,6 +375,10 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
     const int act = bf16 ? 2 : 4;
     const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter, E = cf.num_experts;
     const int gemm_kernels = c.simt ? 2 : 1;  // SIMT launches one kernel per problem
+    // exact re-rounding of z (tensor-core path, bf16 mode): fc1 writes fp32 z into the expert
+    // output buffer, which is free until the expert down GEMM, and the near-midpoint list goes
+    // into the expert activation buffer, free until the expert up GEMM
+    const bool zcheck = bf16 && !c.simt && h->zcheck_delta > 0.f;
     // GEMM operand x: bf16 x as given, fp32 x rounded to bf16 (bf16 mode) or fp32 x (validation mode).
     const void* xa = x;
     bool xa_f32 = cf.x_dtype == LMOE_FP32;
@@ -383,7 +389,8 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         xa_f32 = false;
     }
     {
-        GemmProblem pr[2] = {make_problem(0, p.T, L, bf16 ? EPI_BF16 : EPI_F32, ws_c + p.z, L),
+        GemmProblem pr[2] = {make_problem(0, p.T, L, bf16 && !zcheck ? EPI_BF16 : EPI_F32, ws_c + (zcheck ? p.o : p.z),
+                                          L),
                              make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is)};
         pr[0].kdim[0] = H;
         pr[1].kdim[0] = H;
@@ -394,6 +401,17 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         Operand a[2][2] = {{{xa, p.T}, {nullptr, 0}}, {{xa, p.T}, {nullptr, 0}}};
         Operand b[2][2] = {{{h->w.fc1_w, L}, {nullptr, 0}}, {{h->w.shared_up_w, Is}, {nullptr, 0}}};
         LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
+    }
+    if (zcheck) {
+        const long long cap_ll = std::min<long long>((long long)p.T * L, (long long)p.A * cf.expert_inter * act / 8);
+        const int cap = (int)std::min<long long>(cap_ll, 0x7FFFFFFF);
+        int2* list = reinterpret_cast<int2*>(ws_c + p.aperm);
+        int* count = &reinterpret_cast<WsStats*>(ws_c + p.stats)->zflagged;
+        uint16_t* z = reinterpret_cast<uint16_t*>(ws_c + p.z);
+        LMOE_LAUNCH(1, launch_z_round_flag(reinterpret_cast<const float*>(ws_c + p.o), z, p.T, L, h->zcheck_delta,
+                                           list, cap, count, c.s));
+        LMOE_LAUNCH(1, launch_z_recheck(static_cast<const uint16_t*>(xa), static_cast<const uint16_t*>(h->w.fc1_w),
+                                        H, list, count, cap, z, L, c.s));
     }
     mark(c, 2);
     LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
@@ -671,6 +689,10 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
             if (v < 0 || v > 100000000) return LMOE_ERR_INVALID_ARG;
             h->flag_delta = (float)(v * 1e-9);
             return LMOE_OK;
+        case LMOE_OPT_Z_RECHECK_DELTA:
+            if (v < 0 || v > 100000000) return LMOE_ERR_INVALID_ARG;
+            h->zcheck_delta = (float)(v * 1e-9);
+            return LMOE_OK;
         case LMOE_OPT_SPIN_LIMIT:
             if (v < 1 || v > 0xFFFFFFFFLL) return LMOE_ERR_INVALID_ARG;
             h->spin_limit = (unsigned)v;
@@ -689,6 +711,7 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
     out->device_error = st.device_error;
     out->kernel_launches = h->launches;
     out->cuda_error = h->last_cuda_error;
+    out->z_rechecked = st.zflagged;
     return LMOE_OK;
 }
 

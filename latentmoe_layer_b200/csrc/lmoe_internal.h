@@ -23,7 +23,8 @@ struct WsStats {
     int distinct;       // experts with at least one token
     int max_count;      // largest per-expert count
     int device_error;   // lmoe_status from a device check
-    int pad[60];
+    int zflagged;       // z elements listed for the exact re-rounding
+    int pad[59];
 };
 
 // Epilogue kinds of the GEMM kernels.
@@ -105,6 +106,10 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
 cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts, int* offsets, int* pfx128, int* pfx64,
                               int* pfxdec, int* pfx256, int4* rec32, int4* rec64, int4* rec128, int4* rec256,
                               WsStats* st, cudaStream_t s);
+cudaError_t launch_z_round_flag(const float* z32, uint16_t* z, int rows, int L, float delta, int2* list, int cap,
+                                int* count, cudaStream_t s);
+cudaError_t launch_z_recheck(const uint16_t* x, const uint16_t* w, int K, const int2* list, const int* count, int cap,
+                             uint16_t* z, int L, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* offsets_E,
                                int row_bytes, cudaStream_t s);
 cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,

@@ -168,6 +168,10 @@ def test_call_errors_leave_outputs_untouched(lib):
     assert bool((y == 7.0).all())
     assert lm.latentmoe_set_option(layer.h, 0, 9) == lm.LMOE_ERR_INVALID_ARG
     assert lm.latentmoe_set_option(layer.h, 3, 0) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, -1) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 100000001) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 0) == lm.LMOE_OK
+    assert lm.latentmoe_set_option(layer.h, 5, 0) == lm.LMOE_ERR_INVALID_ARG
 
 
 @pytest.mark.gpu
@@ -206,3 +210,17 @@ def test_profile_events_must_exist(lib):
     assert evs[0].elapsed_time(evs[7]) > 0
     assert lm.latentmoe_set_profile_events(layer.h, None, 0) == lm.LMOE_OK
     layer.close()
+
+
+def test_binding_matches_header_stats_and_options():
+    """The ctypes view of lmoe_stats and the option ids equal the header's."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "latentmoe.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\} lmoe_stats;", hdr).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"int\s+(\w+)\s*;", body)
+    assert fields == [f for f, _ in lm.lmoe_stats._fields_]
+    opts = dict((k, int(v)) for k, v in re.findall(r"LMOE_OPT_(\w+)\s*=\s*(\d+)", hdr))
+    assert opts == {"GEMM_PATH": lm.OPT_GEMM_PATH, "ROUTER_FP64_ALL": lm.OPT_ROUTER_FP64_ALL,
+                    "FLAG_DELTA": lm.OPT_FLAG_DELTA, "SPIN_LIMIT": lm.OPT_SPIN_LIMIT,
+                    "Z_RECHECK_DELTA": lm.OPT_Z_RECHECK_DELTA}
