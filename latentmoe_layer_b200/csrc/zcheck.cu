@@ -12,7 +12,8 @@
 //   2. k_round_flag rounds every element to bf16 (nearest-even) and appends the
 //      elements within `delta` of a rounding midpoint to a list;
 //   3. k_recheck recomputes each listed element as an fp64 sum of the exact
-//      bf16 x bf16 products and stores its nearest-even bf16 rounding.
+//      bf16 x bf16 products (each formed exactly in fp32) and stores its
+//      nearest-even bf16 rounding.
 // The result equals the exactly rounded z whenever the fp32 error is below
 // delta, and the set of listed elements, hence z, is deterministic.
 #include <cuda_bf16.h>
@@ -113,11 +114,12 @@ __global__ void __launch_bounds__(256) k_recheck(const uint16_t* __restrict__ x,
         for (int k = lane; k < K8; k += 32) {
             const uint4 a = __ldg(xr + k), b = __ldg(wr + k);
             const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            // a bf16 x bf16 product has at most 16 significant bits, so the fp32 product is exact
+            // (unless it falls below fp32's normal range); one conversion per product, not two
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                acc = fma((double)__uint_as_float(av[j] << 16), (double)__uint_as_float(bv[j] << 16), acc);
-                acc = fma((double)__uint_as_float(av[j] & 0xFFFF0000u), (double)__uint_as_float(bv[j] & 0xFFFF0000u),
-                          acc);
+                acc += (double)(__uint_as_float(av[j] << 16) * __uint_as_float(bv[j] << 16));
+                acc += (double)(__uint_as_float(av[j] & 0xFFFF0000u) * __uint_as_float(bv[j] & 0xFFFF0000u));
             }
         }
 #pragma unroll
