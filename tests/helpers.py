@@ -9,14 +9,13 @@ import synth
 BF16_MAXABS = 2e-2      # stated bound (bf16 operands, fp32 accumulation)
 BF16_RELFRO = 1e-2
 FP32_RELFRO = 1e-5
-# At Nano/Ultra width the stated 2e-2 max-abs is below what fp32 accumulation
-# can reach against an exactly rounding fp64 reference: fp32-level differences
-# flip ~0.02% of the bf16 roundings of z and of the expert activations, each
-# flip nudges all L entries of the token's weighted sum, and 2-5% of those
-# land on the other side of their bf16 rounding point; the output then moves
-# by ~sqrt(#flips) * ulp(comb) * |W_fc2| ~ 6e-3 rms, 0.02-0.035 at the tail.
-# An IEEE round-to-nearest fp32 path shows the same figures. Wide shapes are
-# therefore held to this derived bound (rel-Frobenius stays at the stated 1e-2).
+# Bound for the IEEE fp32 SIMT validation kernels at Nano/Ultra width only. Plain
+# fp32 accumulation flips ~0.02% of the bf16 roundings of z and of the expert
+# activations against an exactly rounding fp64 reference. A flipped z element
+# moves all k expert outputs of its token, and the output then moves by
+# 0.02-0.035 at the tail. The tensor-core paths re-round z exactly and meet the
+# stated 2e-2. The SIMT kernels do not re-round z, so they are held to this
+# derived bound; rel-Frobenius stays at the stated 1e-2.
 BF16_MAXABS_WIDE = 5e-2
 
 

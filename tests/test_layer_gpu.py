@@ -42,7 +42,9 @@ def run_and_compare(shape, mode=0, path=GEMM_AUTO, full=True):
     yg = y.cpu().numpy()
     if mode == 1:
         return H.assert_fp32_close(yg, yref), layer
-    return H.assert_bf16_close(yg, yref, wide=H.is_wide(shape)), layer
+    # the stated 2e-2 max-abs everywhere on the tensor-core paths (z is re-rounded exactly); the IEEE
+    # fp32 SIMT validation kernels have no z re-rounding and keep the derived allowance at full width
+    return H.assert_bf16_close(yg, yref, wide=H.is_wide(shape) and path == GEMM_SIMT), layer
 
 
 @pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_SIMT])
@@ -155,7 +157,7 @@ def _sampled_parity(shape, rows, route_rows, path=GEMM_AUTO):
     wts = H.host_weights_for(shape, dev, experts)
     yref, iref, _ = H.oracle_forward(shape, H.host_x(shape, dev, rows), wts)
     assert np.array_equal(iref, gi[rows])
-    ma, rf = H.assert_bf16_close(y.cpu().numpy()[rows], yref, wide=True)
+    ma, rf = H.assert_bf16_close(y.cpu().numpy()[rows], yref)
     hot = float(gc[:16].sum()) / gc.sum()
     print("%s max_abs=%.3g rel_fro=%.3g flagged=%d distinct=%d max_count=%d hot16_share=%.3f" %
           (shape.name, ma, rf, st.flagged_tokens, st.distinct_experts, st.max_expert_tokens, hot))
@@ -253,5 +255,5 @@ def test_pre_norm_residual_block(shape, path):
     host = synth.host_inputs(shape)
     yref, iref, _ = oracle.forward_block(oracle.make_cfg(shape), host["x"], H.bf16_to_bits(g), 1e-5, host)
     assert np.array_equal(idx.cpu().numpy(), iref)
-    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref, wide=H.is_wide(shape))
+    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref)
     print("block %s path=%d max_abs=%.3g rel_fro=%.3g" % (shape.name, path, ma, rf))
