@@ -26,8 +26,10 @@
  *
  * Modes: LMOE_MODE_BF16 feeds bf16 operands to tensor-core GEMMs with fp32
  * accumulation (z, the expert activations, the weighted sum and the shared
- * activations are rounded to bf16 as GEMM operands); LMOE_MODE_FP32 is a
- * validation mode with fp32 operands and no intermediate rounding.
+ * activations are rounded to bf16 as GEMM operands; z, which every routed
+ * expert of a token reads, is rounded exactly: see LMOE_OPT_Z_RECHECK_DELTA);
+ * LMOE_MODE_FP32 is a validation mode with fp32 operands and no intermediate
+ * rounding.
  *
  * Errors: every argument is validated before anything is launched; on
  * LMOE_ERR_INVALID_ARG / _WORKSPACE / _UNSUPPORTED no output is touched. The
