@@ -256,7 +256,9 @@ typedef struct {
     int kernel_launches;    /* kernels the last route/forward call on the handle launched */
     int cuda_error;         /* cudaError_t of the last CUDA runtime call on the handle that
                                failed (a call that returned LMOE_ERR_CUDA), 0 if none     */
-    int z_rechecked;        /* z elements re-rounded exactly (LMOE_OPT_Z_RECHECK_DELTA)    */
+    int z_rechecked;        /* z elements listed for exact re-rounding (LMOE_OPT_Z_RECHECK_DELTA);
+                               all are re-rounded unless the count exceeds the list's room,
+                               min(T*L, T*top_k*expert_inter/4) entries                  */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */
