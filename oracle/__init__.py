@@ -56,6 +56,8 @@ def _get():
         lib.lmo_select.argtypes = [vp, vp, vp]
         lib.lmo_logits.argtypes = [vp, vp, vp, i64, vp]
         lib.lmo_route.argtypes = [vp, vp, vp, vp, i64, vp, vp]
+        lib.lmo_latent.argtypes = [vp, vp, vp, i64, vp]
+        lib.lmo_latent.restype = ctypes.c_int
         lib.lmo_forward.argtypes = [vp, vp, vp, i64, vp, vp, vp]
         lib.lmo_update_bias.argtypes = [ctypes.c_int, vp, vp, ctypes.c_double, vp, vp]
         lib.lmo_rmsnorm.argtypes = [ctypes.c_int, vp, vp, ctypes.c_double, i64, vp]
@@ -117,6 +119,16 @@ def logits(cfg: LmoCfg, x, router_w) -> np.ndarray:
     n = x.shape[0]
     out = np.zeros((n, cfg.E), dtype=np.float64)
     _get().lmo_logits(ctypes.byref(cfg), x.ctypes.data, rw.ctypes.data, n, out.ctypes.data)
+    return out
+
+
+def latent(cfg: LmoCfg, x, fc1_w) -> np.ndarray:
+    """fc1_latent_proj of the rows of x before its bf16 rounding (fp64 [n, L])."""
+    x = _xarr(cfg, x)
+    w = _c(fc1_w, np.uint16)
+    n = x.shape[0]
+    out = np.zeros((n, cfg.L), dtype=np.float64)
+    _get().lmo_latent(ctypes.byref(cfg), x.ctypes.data, w.ctypes.data, n, out.ctypes.data)
     return out
 
 

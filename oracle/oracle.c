@@ -158,6 +158,23 @@ int lmo_route(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, const
     return bad ? -1 : 0;
 }
 
+/* fc1_latent_proj of n tokens, unrounded ("Nemotron 3 Ultra 架构 QA", Q5.1). */
+int lmo_latent(const lmo_cfg* cfg, const void* x, const uint16_t* fc1_w, int64_t n, double* out) {
+    const int H = cfg->H, L = cfg->L;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < n; ++t) {
+        double* xh = (double*)malloc(sizeof(double) * (size_t)H);
+        for (int h = 0; h < H; ++h) xh[h] = rho(cfg, x_at(cfg, x, t, h));
+        for (int l = 0; l < L; ++l) {
+            double s = 0.0;
+            for (int h = 0; h < H; ++h) s += xh[h] * bf(fc1_w[(int64_t)l * H + h]);
+            out[t * L + l] = s;
+        }
+        free(xh);
+    }
+    return 0;
+}
+
 /* Full layer for each token ("Nemotron 3 Ultra 架构 QA", Q5.1 and Q5.7):
  *   z    = rho(x^ W_fc1^T)                       fc1_latent_proj, H -> L
  *   a_e  = rho(relu(z W_up[e]^T)^2)              expert up + relu2 (Q2.6)

@@ -77,6 +77,11 @@ int lmo_logits(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, int6
 int lmo_route(const lmo_cfg* cfg, const void* x, const uint16_t* router_w, const float* e_bias, int64_t n,
               int32_t* idx, double* w);
 
+/* fc1_latent_proj before its rounding ("Nemotron 3 Ultra 架构 QA", Q5.1; the
+ * step z = rho(x^ W_fc1^T) of lmo_forward without rho): out[t, l] =
+ * sum_h rho(x[t, h]) W_fc1[l, h] in fp64, for n tokens. */
+int lmo_latent(const lmo_cfg* cfg, const void* x, const uint16_t* fc1_w, int64_t n, double* out);
+
 /* Full layer for n tokens. x holds those n rows; y[n, H] fp64. idx/w may be NULL. */
 int lmo_forward(const lmo_cfg* cfg, const void* x, const lmo_weights* wts, int64_t n, int32_t* idx, double* w,
                 double* y);
