@@ -151,6 +151,31 @@ def test_logits_one_hot_picks_router_column(built_oracle):
     assert np.array_equal(lg, bits_to_f64(wr).T)
 
 
+def test_latent_one_hot_picks_fc1_column(built_oracle):
+    w = small_shape()
+    cfg = built_oracle.make_cfg(w)
+    w1 = synth.host_tensor(w, "fc1_w", 1)
+    x = np.zeros((w.H, w.H), dtype=np.float32)
+    np.fill_diagonal(x, 1.0)
+    assert np.array_equal(built_oracle.latent(cfg, x, w1), bits_to_f64(w1).T)
+
+
+@pytest.mark.parametrize("x_f32", [True, False])
+def test_latent_is_the_matmul_of_the_rounded_input(built_oracle, x_f32):
+    """bf16 mode: z before its rounding is rho(x) W_fc1^T (numpy fp64 matmul); with
+    bf16 x the rounding of x is the identity."""
+    w = small_shape(x_f32=x_f32, H=256, L=64, T=9)
+    cfg = built_oracle.make_cfg(w)
+    inp = inputs(w)
+    x = inp["x"]
+    xr = f32_to_bf16_bits(x) if x_f32 else x
+    ref = bits_to_f64(xr) @ bits_to_f64(inp["fc1_w"]).T
+    got = built_oracle.latent(cfg, x, inp["fc1_w"])
+    assert np.allclose(got, ref, rtol=1e-13, atol=1e-13)
+    if x_f32:  # rho(x) is applied: the unrounded x gives a different product
+        assert not np.allclose(got, x.astype(np.float64) @ bits_to_f64(inp["fc1_w"]).T, rtol=1e-9, atol=0)
+
+
 def test_weights_sum_to_scale(built_oracle):
     w = replace(TINY, T=64)
     cfg = built_oracle.make_cfg(w)
