@@ -242,7 +242,9 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
     # End to end through the public call with host buffers: every step copies its
     # x from pinned host memory to the device, runs the layer and copies y back.
     # Copies run on their own streams, double-buffered, so step i's compute
-    # overlaps step i+1's upload and step i-1's download (as a serving loop would).
+    # overlaps step i+1's upload and step i-1's download (as a serving loop would):
+    # pipelined throughput. e2e_serial_run times the same steps with each step's
+    # upload, forward and download in sequence on one stream (per-call latency).
     xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     xh.copy_(x)
     yh = torch.empty((shape.T, shape.H), dtype=torch.float32, pin_memory=True)
@@ -280,13 +282,29 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
         torch.cuda.synchronize()
         return start.elapsed_time(end)
 
+    def e2e_serial_run(n):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        for i in range(n):
+            xd[0].copy_(xh, non_blocking=True)
+            layer.forward(xd[0], yd[0])
+            yh.copy_(yd[0], non_blocking=True)
+        end.record(comp)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
     e2e_run(max(2, warmup))
     e_steps = max(2, min(steps, 50))
     if dist is not None:
         dist.barrier()
     e_ms = max_over_ranks(e2e_run(e_steps), dist, "cuda")
+    e2e_serial_run(2)
+    if dist is not None:
+        dist.barrier()
+    es_ms = max_over_ranks(e2e_serial_run(e_steps), dist, "cuda")
     res = {
-        "ms": ms, "stage_ms": stage_ms, "stats": st, "loads": loads, "clocks": clk, "e2e_ms": e_ms,
+        "ms": ms, "stage_ms": stage_ms, "stats": st, "loads": loads, "clocks": clk, "e2e_ms": e_ms, "e2e_serial_ms": es_ms,
         "e2e_steps": e_steps,
         "h2d": x.numel() * x.element_size(), "d2h": y.numel() * 4, "layer": layer, "dev": dev,
     }
@@ -308,10 +326,10 @@ def roofline_for(shape, res, peaks, peak_src, prefill: bool, nvfp4=False):
     name, kms = ("expert_up_gemm", up_ms) if up_ms >= dn_ms else ("expert_down_gemm", dn_ms)
     if prefill:
         ach = flops / (kms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        peak = peaks["bf16_tflops"]
         return {"kernel": name, "bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ach / peak, 4), "peak_kind": "%s sustained bf16" % peak_src,
-                "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                "frac": round(ach / peak, 4), "peak_kind": "%s burst bf16 (the target denominator)" % peak_src,
+                "frac_of_sustained_peak": round(ach / peaks["bf16_tflops_sustained"], 4),
                 "traffic": (round(UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT * shape.T * shape.k)
                             if name == "expert_up_gemm" and UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT else None),
                 "traffic_note": "ncu capture of the same kernel on probe_e64, scaled by assignments",
@@ -321,6 +339,14 @@ def roofline_for(shape, res, peaks, peak_src, prefill: bool, nvfp4=False):
     return {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
             "frac": round(ach / peak, 4), "peak_kind": "%s HBM copy" % peak_src, "traffic": None,
             "algorithmic_per_launch": byts, "launch_ms": round(kms, 4)}
+
+
+def target_of(shape, summary, prefill):
+    """The layer-level target the throughput is held to: >= 60% of the bf16 tensor
+    peak (burst) at large token counts, >= 70% of HBM bandwidth over the touched
+    weights at decode sizes."""
+    key, goal = ("layer_frac_of_burst_bf16", 0.60) if prefill else ("layer_frac_of_hbm", 0.70)
+    return {"metric": key, "value": summary[key], "target": goal, "met": bool(summary[key] >= goal)}
 
 
 def layer_summary(shape, res, peaks, peak_src, steps, nvfp4=False):
@@ -441,10 +467,14 @@ def run_ours(args):
                    "l2": l2_note(shape)},
         "roofline": roofline_for(shape, res, peaks, peak_src, prefill, nvfp4=nv),
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
-                "d2h_bytes_per_step": res["d2h"]},
+                "d2h_bytes_per_step": res["d2h"],
+                "mode": "pipelined: pinned-host copies double-buffered on their own streams, overlapping compute",
+                "serial_value": round(world * shape.T * res["e2e_steps"] / (res["e2e_serial_ms"] * 1e-3), 1),
+                "serial_mode": "each step's upload, forward and download in sequence on one stream"},
         "gpu_launches": res["stats"].kernel_launches * args.steps,
         "clocks": res["clocks"],
         "layer": summary,
+        "target": target_of(shape, summary, prefill),
     }
     layer, dev = res["layer"], res["dev"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not nv:
@@ -462,6 +492,7 @@ def run_ours(args):
                              "roofline": roofline_for(s2, r2, peaks, peak_src, s2.T * s2.k > 64 * s2.E),
                              "layer": layer_summary(s2, r2, peaks, peak_src, args.secondary_steps),
                              "clocks": r2["clocks"]}
+        line["secondary"]["target"] = target_of(s2, line["secondary"]["layer"], s2.T * s2.k > 64 * s2.E)
         r2["layer"].close()
         del r2
         torch.cuda.empty_cache()
@@ -475,6 +506,7 @@ def run_ours(args):
             "roofline": roofline_for(s3, r3, peaks, peak_src, s3.T * s3.k > 64 * s3.E, nvfp4=True),
             "layer": layer_summary(s3, r3, peaks, peak_src, args.secondary_steps, nvfp4=True),
             "clocks": r3["clocks"]}
+        line["nvfp4_experts"]["target"] = target_of(s3, line["nvfp4_experts"]["layer"], s3.T * s3.k > 64 * s3.E)
         r3["layer"].close()
     if rank == 0:
         print(json.dumps(line))

@@ -27,7 +27,9 @@
  * Modes: LMOE_MODE_BF16 feeds bf16 operands to tensor-core GEMMs with fp32
  * accumulation (z, the expert activations, the weighted sum and the shared
  * activations are rounded to bf16 as GEMM operands; z, which every routed
- * expert of a token reads, is rounded exactly: see LMOE_OPT_Z_RECHECK_DELTA);
+ * expert of a token reads, is re-rounded so that it equals the exact rounding
+ * of x W_fc1^T whenever the fp32 error of an element is below the margin of
+ * LMOE_OPT_Z_RECHECK_DELTA);
  * LMOE_MODE_FP32 is a validation mode with fp32 operands and no intermediate
  * rounding.
  *
@@ -234,7 +236,12 @@ typedef enum {
                                     tokens at decode sizes, else 128); the option then applies to
                                     the dense GEMMs, and 3 is unsupported (LMOE_ERR_UNSUPPORTED). */
     LMOE_OPT_ROUTER_FP64_ALL = 1,/* 1: every token's logits recomputed in fp64 (validation)      */
-    LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin for the fp64 re-check, in 1e-9 units        */
+    LMOE_OPT_FLAG_DELTA = 2,     /* near-edge margin delta of the fp64 re-check, in 1e-9 units
+                                    (default 20000 = 2e-5): a token is re-decided from exact
+                                    fp64 logits when its k-th / (k+1)-th fp32 choice-score gap
+                                    is within 1e-6 + delta (group scores: 1e-6 + 2 delta); the
+                                    routing is exact whenever every fp32 choice score is within
+                                    delta / 2 of its exact value                               */
     LMOE_OPT_SPIN_LIMIT = 3,     /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */
     LMOE_OPT_Z_RECHECK_DELTA = 4 /* margin of the exact re-rounding of z, in 1e-9 units (default
                                     5000 = 5e-6; 0 disables). bf16 mode, tensor-core GEMMs: the
@@ -256,13 +263,27 @@ typedef struct {
     int kernel_launches;    /* kernels the last route/forward call on the handle launched */
     int cuda_error;         /* cudaError_t of the last CUDA runtime call on the handle that
                                failed (a call that returned LMOE_ERR_CUDA), 0 if none     */
-    int z_rechecked;        /* z elements listed for exact re-rounding (LMOE_OPT_Z_RECHECK_DELTA);
-                               all are re-rounded unless the count exceeds the list's room,
-                               min(T*L, T*top_k*expert_inter/4) entries                  */
+    int z_rechecked;        /* z elements listed and re-rounded exactly (LMOE_OPT_Z_RECHECK_DELTA);
+                               the list has room for all T*L elements                    */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */
 lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out);
+
+/* Byte offsets, from the start of a call's workspace, of intermediate buffers
+ * that tests and tools read back after a call on T tokens (a diagnostic: the
+ * layout may change between versions). logits_f32 [T, E] fp32 router logits
+ * (latentmoe_route/forward); z_f32 [T, L] fp32 fc1 product before rounding
+ * (bf16 mode with z re-rounding on, valid after latentmoe_ep_front: a forward
+ * overwrites it with the expert outputs); z [T, L] bf16 latent after
+ * re-rounding; flag_list: int32 ids of the tokens re-decided in fp64
+ * (lmoe_stats.flagged_tokens of them); perm [T*k] int32: token of each row in
+ * expert order; slot [T, k] int32: row in expert order of each (token, j);
+ * total = latentmoe_workspace_size(T). */
+typedef struct {
+    size_t logits_f32, z_f32, z, flag_list, perm, slot, total;
+} lmoe_ws_layout;
+lmoe_status latentmoe_workspace_layout(const lmoe_handle* h, int T, lmoe_ws_layout* out);
 
 /* Routing for callers that cannot allocate device memory (a real-time or
  * latency-critical section where cudaMalloc's implicit synchronisation is not

@@ -7,7 +7,10 @@ convenience wrapper that owns a handle and a workspace.
 
 Importing this package does not load the library; the first call does, and it
 raises ``RuntimeError`` if liblatentmoe.so has not been built (there is no
-fallback implementation).
+fallback implementation). With ``LATENTMOE_CHECKS=1`` in the environment the
+checking build (liblatentmoe_checks.so: device-side bounds checks that report
+LMOE_ERR_INVALID_ARG instead of touching memory out of range) is loaded instead;
+``LATENTMOE_LIB=<path>`` loads that build of the library.
 """
 from __future__ import annotations
 
@@ -15,7 +18,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblatentmoe.so")
+LIB_PATH = os.environ.get("LATENTMOE_LIB") or os.path.join(
+    _HERE, "liblatentmoe_checks.so" if os.environ.get("LATENTMOE_CHECKS") == "1" else "liblatentmoe.so")
 
 LMOE_OK, LMOE_ERR_INVALID_ARG, LMOE_ERR_UNSUPPORTED, LMOE_ERR_WORKSPACE, LMOE_ERR_CUDA, LMOE_ERR_TIMEOUT, \
     LMOE_ERR_INTERNAL = range(7)
@@ -29,7 +33,7 @@ EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "l
            "latentmoe_destroy", "latentmoe_status_string", "latentmoe_set_option", "latentmoe_read_stats",
            "latentmoe_selftest_bounded_wait", "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias", "latentmoe_forward_block",
            "latentmoe_quantize_nvfp4", "latentmoe_ep_front", "latentmoe_ep_workspace_size", "latentmoe_ep_experts",
-           "latentmoe_ep_back"]
+           "latentmoe_ep_back", "latentmoe_workspace_layout"]
 
 
 class lmoe_config(ctypes.Structure):
@@ -50,6 +54,10 @@ class lmoe_stats(ctypes.Structure):
     _fields_ = [("flagged_tokens", ctypes.c_int), ("distinct_experts", ctypes.c_int),
                 ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int),
                 ("kernel_launches", ctypes.c_int), ("cuda_error", ctypes.c_int), ("z_rechecked", ctypes.c_int)]
+
+
+class lmoe_ws_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("logits_f32", "z_f32", "z", "flag_list", "perm", "slot", "total")]
 
 
 class LmoeError(RuntimeError):
@@ -91,11 +99,13 @@ def load():
     lib.latentmoe_ep_workspace_size.argtypes = [vp, i32, i32, ctypes.POINTER(sz)]
     lib.latentmoe_ep_experts.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
     lib.latentmoe_ep_back.argtypes = [vp, vp, i32, vp, vp, sz, vp]
+    lib.latentmoe_workspace_layout.argtypes = [vp, i32, ctypes.POINTER(lmoe_ws_layout)]
     for f in ("latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
               "latentmoe_set_option", "latentmoe_read_stats", "latentmoe_selftest_bounded_wait",
               "latentmoe_set_profile_events", "latentmoe_route_noalloc", "latentmoe_update_bias",
               "latentmoe_forward_block", "latentmoe_quantize_nvfp4", "latentmoe_ep_front",
-              "latentmoe_ep_workspace_size", "latentmoe_ep_experts", "latentmoe_ep_back"):
+              "latentmoe_ep_workspace_size", "latentmoe_ep_experts", "latentmoe_ep_back",
+              "latentmoe_workspace_layout"):
         getattr(lib, f).restype = i32
     _lib = lib
     return lib
@@ -180,6 +190,12 @@ def quantize_nvfp4(w):
     if s != LMOE_OK:
         raise LmoeError(s, "latentmoe_quantize_nvfp4")
     return codes, sf, gs
+
+
+def latentmoe_workspace_layout(h, T: int):
+    out = lmoe_ws_layout()
+    s = load().latentmoe_workspace_layout(h, T, ctypes.byref(out))
+    return s, out
 
 
 def latentmoe_selftest_bounded_wait(h) -> int:
@@ -313,6 +329,20 @@ class LatentMoE:
         s = latentmoe_update_bias(self.h, _p(counts), _p(b), float(eta), _p(b), _p(maxvio), self._stream())
         if s != LMOE_OK:
             raise LmoeError(s, "latentmoe_update_bias")
+
+    def layout(self, T: int):
+        s, out = latentmoe_workspace_layout(self.h, T)
+        if s != LMOE_OK:
+            raise LmoeError(s, "latentmoe_workspace_layout")
+        return out
+
+    def ws_view(self, offset: int, shape, dtype):
+        """A tensor view of the workspace at a byte offset (diagnostics)."""
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * self.torch.empty((), dtype=dtype).element_size()
+        return self._ws[offset:offset + nbytes].view(dtype).view(*shape)
 
     def stats(self):
         s, st = latentmoe_read_stats(self.h, _p(self._ws))

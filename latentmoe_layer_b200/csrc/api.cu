@@ -112,6 +112,10 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     p.o = take(A * L * 4);
     p.comb = take((size_t)T * L * act);
     p.as = take((size_t)T * Is * act);
+    // near-midpoint list of the exact z re-rounding, room for every element of z: it
+    // shares the expert activation buffer (free until the expert up GEMM) when that
+    // is large enough (top_k * I >= 4 L), else it has its own
+    p.zlist = (A * I * act >= (size_t)T * L * 8) ? p.aperm : take((size_t)T * L * 8);
     p.total = off;
     return true;
 }
@@ -141,6 +145,7 @@ lmoe_status check_config(const lmoe_config* c) {
     if (c->n_group > 1 && c->num_experts / c->n_group < 2) return LMOE_ERR_UNSUPPORTED;
     if (c->hidden > 16384) return LMOE_ERR_UNSUPPORTED;  // fp64 router stages one x row in shared memory
     if ((long long)c->max_tokens * c->top_k > (1LL << 30)) return LMOE_ERR_UNSUPPORTED;
+    if ((long long)c->max_tokens * c->latent > 0x7FFFFFFFLL) return LMOE_ERR_UNSUPPORTED;  // z element list index
     return LMOE_OK;
 }
 
@@ -326,7 +331,7 @@ lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int3
     LMOE_LAUNCH(3, launch_permute(h, p, ws, counts_out, c.s));
     LMOE_LAUNCH((idx_out || w_out) ? 1 : 0,
                 launch_copy_routing(reinterpret_cast<const int*>(ws + p.idx), reinterpret_cast<const float*>(ws + p.wgt),
-                                    idx_out, w_out, (long long)p.T * cf.top_k, c.s));
+                                    idx_out, w_out, (long long)p.T * cf.top_k, h->num_sms, c.s));
     return LMOE_OK;
 }
 
@@ -375,16 +380,16 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
     const int act = bf16 ? 2 : 4;
     const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter, E = cf.num_experts;
     const int gemm_kernels = c.simt ? 2 : 1;  // SIMT launches one kernel per problem
-    // exact re-rounding of z (tensor-core path, bf16 mode): fc1 writes fp32 z into the expert
+    // exact re-rounding of z (bf16 mode, every GEMM path): fc1 writes fp32 z into the expert
     // output buffer, which is free until the expert down GEMM, and the near-midpoint list goes
-    // into the expert activation buffer, free until the expert up GEMM
-    const bool zcheck = bf16 && !c.simt && h->zcheck_delta > 0.f;
+    // into the plan's list buffer (room for all of z, so no element can be left out)
+    const bool zcheck = bf16 && h->zcheck_delta > 0.f;
     // GEMM operand x: bf16 x as given, fp32 x rounded to bf16 (bf16 mode) or fp32 x (validation mode).
     const void* xa = x;
     bool xa_f32 = cf.x_dtype == LMOE_FP32;
     if (bf16 && cf.x_dtype == LMOE_FP32) {
         LMOE_LAUNCH(1, launch_convert_x(static_cast<const float*>(x), reinterpret_cast<uint16_t*>(ws_c + p.xbf),
-                                        (long long)p.T * H, c.s));
+                                        (long long)p.T * H, h->num_sms, c.s));
         xa = ws_c + p.xbf;
         xa_f32 = false;
     }
@@ -403,19 +408,18 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
     }
     if (zcheck) {
-        const long long cap_ll = std::min<long long>((long long)p.T * L, (long long)p.A * cf.expert_inter * act / 8);
-        const int cap = (int)std::min<long long>(cap_ll, 0x7FFFFFFF);
-        int2* list = reinterpret_cast<int2*>(ws_c + p.aperm);
+        const int cap = (int)std::min<long long>((long long)p.T * L, 0x7FFFFFFF);  // T * L < 2^31 (create)
+        int2* list = reinterpret_cast<int2*>(ws_c + p.zlist);
         int* count = &reinterpret_cast<WsStats*>(ws_c + p.stats)->zflagged;
         uint16_t* z = reinterpret_cast<uint16_t*>(ws_c + p.z);
         LMOE_LAUNCH(1, launch_z_round_flag(reinterpret_cast<const float*>(ws_c + p.o), z, p.T, L, h->zcheck_delta,
-                                           list, cap, count, c.s));
+                                           list, cap, count, h->num_sms, c.s));
         LMOE_LAUNCH(1, launch_z_recheck(static_cast<const uint16_t*>(xa), static_cast<const uint16_t*>(h->w.fc1_w),
-                                        H, list, count, cap, z, L, c.s));
+                                        H, p.T, c.err, list, count, cap, z, L, h->num_sms, c.s));
     }
     mark(c, 2);
-    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
-                                      reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, c.s));
+    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, p.T, c.err, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
+                                      reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, h->num_sms, c.s));
     mark(c, 3);
     return LMOE_OK;
 }
@@ -482,8 +486,8 @@ lmoe_status stage_back(Ctx& c, const float* o, float* y, const uint16_t* resid) 
     char* ws_c = c.ws;
     const bool bf16 = cf.mode == LMOE_MODE_BF16;
     const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter;
-    LMOE_LAUNCH(1, launch_combine(o, reinterpret_cast<const int*>(ws_c + p.slot), ws_c + p.comb, p.T, cf.top_k, L,
-                                  bf16, c.s));
+    LMOE_LAUNCH(1, launch_combine(o, p.A, c.err, reinterpret_cast<const int*>(ws_c + p.slot), ws_c + p.comb, p.T,
+                                  cf.top_k, L, bf16, h->num_sms, c.s));
     mark(c, 6);
     {
         GemmProblem pr = make_problem(0, p.T, H, EPI_F32, y, H);
@@ -513,7 +517,7 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
     h->launches = 0;
     mark(c, 0);
     if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
-                                                reinterpret_cast<uint16_t*>(const_cast<void*>(x)), c.s));
+                                                reinterpret_cast<uint16_t*>(const_cast<void*>(x)), h->num_sms, c.s));
     s = do_route(c, x, topk_idx, topk_w, expert_counts);
     if (s != LMOE_OK) return s;
     mark(c, 1);
@@ -699,6 +703,20 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
             return LMOE_OK;
     }
     return LMOE_ERR_INVALID_ARG;
+}
+
+lmoe_status latentmoe_workspace_layout(const lmoe_handle* h, int T, lmoe_ws_layout* out) {
+    if (!h || !out || T < 1 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+    Plan p;
+    plan_of(h->cfg, T, p);
+    out->logits_f32 = p.logits;
+    out->z_f32 = p.o;
+    out->z = p.z;
+    out->flag_list = p.flaglist;
+    out->perm = p.perm;
+    out->slot = p.slot;
+    out->total = p.total;
+    return LMOE_OK;
 }
 
 lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stats* out) {

@@ -19,6 +19,7 @@
 #define LMOE_MAX_BN 256
 #endif
 
+
 namespace lmoe {
 namespace {
 
@@ -115,7 +116,14 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         const GemmProblem& pr = P.prob[0];
         const int nct = n_col_tiles(pr, S::kOutCols);
         const int mt = t / nct, ct = t % nct;
-        const int4 rc = __ldg(grouped_records<S::kActRows>(P.r) + mt);
+        int4 rc = __ldg(grouped_records<S::kActRows>(P.r) + mt);
+#if LMOE_CHECKS
+        // a tile record must name a group and a row range inside the permuted rows
+        if (!lmoe_check((unsigned)rc.x < (unsigned)P.r.E && rc.y >= 0 && rc.z >= 1 && rc.z <= S::kActRows &&
+                            rc.y + rc.z <= __ldg(P.r.offsets + P.r.E),
+                        P.err))
+            rc = make_int4(0, 0, 0, 0);  // a tile with no rows: loads stay in bounds, nothing is stored
+#endif
         const int e = pr.expert_mod ? rc.x % pr.expert_mod : rc.x;
         ti.p = 0;
         ti.row0 = rc.y;

@@ -9,7 +9,7 @@ struct lmoe_handle {
     int* derr = nullptr;       // same word, device view
     int gemm_path = 0;         // lmoe_option LMOE_OPT_GEMM_PATH
     int fp64_all = 0;          // LMOE_OPT_ROUTER_FP64_ALL
-    float flag_delta = 3e-6f;  // LMOE_OPT_FLAG_DELTA (measured max |fp32 - fp64| score: 4.5e-7)
+    float flag_delta = 2e-5f;  // LMOE_OPT_FLAG_DELTA (10x the largest fp32 score error seen at Ultra width, x2)
     float zcheck_delta = 5e-6f;  // LMOE_OPT_Z_RECHECK_DELTA (mean |fp32 - exact| of z: ~3e-7)
     unsigned spin_limit = 1u << 24;
     int num_sms = 148;

@@ -6,7 +6,25 @@
 
 #include "../../include/latentmoe.h"
 
+#ifndef LMOE_CHECKS
+#define LMOE_CHECKS 0  // 1: the checking build (device-side bounds checks, see lmoe_check)
+#endif
+
 namespace lmoe {
+
+// Device-side bounds check of the checking build (LMOE_CHECKS=1): a false
+// condition records LMOE_ERR_INVALID_ARG in the call's error word and the
+// caller skips the access it guards. In the default build it is always true
+// and compiles away.
+__device__ __forceinline__ bool lmoe_check(bool ok, int* err) {
+#if LMOE_CHECKS
+    if (!ok) atomicCAS(err, 0, 1);
+    return ok;
+#else
+    (void)err;
+    return true;
+#endif
+}
 
 constexpr int kBM = 128;          // tensor-core tile rows (MMA M)
 constexpr int kBK = 64;           // K elements per pipeline stage (one 128-byte swizzle row of bf16)
@@ -88,7 +106,7 @@ struct DeviceRouting {
 struct Plan {
     size_t total;
     size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64,
-        rec128, rec256, blockcounts, perm, slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as;
+        rec128, rec256, blockcounts, perm, slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as, zlist;
     int T, A, nblk;
 };
 
@@ -97,7 +115,7 @@ struct Plan {
 // ---- launchers (all asynchronous on `stream`; return cudaError_t) ----------
 struct lmoe_handle;
 namespace lmoe {
-cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStream_t s);
+cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, int sms, cudaStream_t s);
 cudaError_t launch_router_select(const lmoe_handle* h, const Plan& p, char* ws, bool fp64_all, cudaStream_t s);
 cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Plan& p, char* ws, bool all,
                                    cudaStream_t s);
@@ -107,19 +125,19 @@ cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts,
                               int* pfxdec, int* pfx256, int4* rec32, int4* rec64, int4* rec128, int4* rec256,
                               WsStats* st, cudaStream_t s);
 cudaError_t launch_z_round_flag(const float* z32, uint16_t* z, int rows, int L, float delta, int2* list, int cap,
-                                int* count, cudaStream_t s);
-cudaError_t launch_z_recheck(const uint16_t* x, const uint16_t* w, int K, const int2* list, const int* count, int cap,
-                             uint16_t* z, int L, cudaStream_t s);
-cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* offsets_E,
-                               int row_bytes, cudaStream_t s);
-cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
-                           cudaStream_t s);
-cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out,
-                           cudaStream_t s);
+                                int* count, int sms, cudaStream_t s);
+cudaError_t launch_z_recheck(const uint16_t* x, const uint16_t* w, int K, int rows, int* err, const int2* list,
+                             const int* count, int cap,
+                             uint16_t* z, int L, int sms, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, int src_rows, int* err, void* dst, const int* perm, int rows_total_max,
+                               const int* offsets_E,
+                               int row_bytes, int sms, cudaStream_t s);
+cudaError_t launch_combine(const float* o, int o_rows, int* err, const int* slot, void* comb, int T, int k, int L,
+                           bool out_bf16, int sms, cudaStream_t s);
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out, int sms, cudaStream_t s);
 cudaError_t launch_update_bias(const int32_t* counts, const float* bias_in, int E, double eta, float* bias_out,
                                double* maxvio, cudaStream_t s);
-cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n,
-                                cudaStream_t s);
+cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n, int sms, cudaStream_t s);
 cudaError_t launch_gemm_simt(const GemmProblem* probs, int nprob, bool a_f32, const DeviceRouting& r, int max_rows,
                              cudaStream_t s);
 cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,

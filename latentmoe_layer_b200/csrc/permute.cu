@@ -19,12 +19,14 @@ namespace {
 
 constexpr int kChunk = 256;  // tokens per counting block
 
-__global__ void k_count(const int32_t* __restrict__ idx, int T, int k, int E, int* __restrict__ blockcounts) {
+__global__ void k_count(const int32_t* __restrict__ idx, int T, int k, int E, int* __restrict__ blockcounts,
+                        int* err) {
     extern __shared__ int hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int t0 = blockIdx.x * kChunk, t1 = min(T, t0 + kChunk);
-    for (int i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x) atomicAdd(&hist[idx[i]], 1);
+    for (int i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x)
+        if (lmoe_check((unsigned)idx[i] < (unsigned)E, err)) atomicAdd(&hist[idx[i]], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) blockcounts[(size_t)blockIdx.x * E + e] = hist[e];
 }
@@ -156,7 +158,7 @@ constexpr int kScatterWarps = 8;
 __global__ void __launch_bounds__(kScatterWarps * 32)
     k_scatter(const int32_t* __restrict__ idx, const float* __restrict__ w, int T, int k, int E,
               const int* __restrict__ blockcounts, const int* __restrict__ offsets, int* __restrict__ perm,
-              int* __restrict__ slot, float* __restrict__ wperm) {
+              int* __restrict__ slot, float* __restrict__ wperm, int* err) {
     extern __shared__ int sm[];
     int* cur = sm;                        // [kScatterWarps][E] per-warp cursors
     int* sidx = sm + kScatterWarps * E;   // [kChunk * k]
@@ -168,7 +170,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
     __syncthreads();
     const int w0 = warp * (kChunk / kScatterWarps);
     const int w1 = min(t1 - t0, w0 + kChunk / kScatterWarps);
-    for (int i = w0 * k + lane; i < w1 * k; i += 32) atomicAdd(&cur[warp * E + sidx[i]], 1);
+    for (int i = w0 * k + lane; i < w1 * k; i += 32)
+        if (lmoe_check((unsigned)sidx[i] < (unsigned)E, err)) atomicAdd(&cur[warp * E + sidx[i]], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {  // exclusive prefix over the warps
         int run = offsets[e] + blockcounts[(size_t)blockIdx.x * E + e];
@@ -183,6 +186,10 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
     for (int tl = w0; tl < w1; ++tl) {
         for (int j = lane; j < k; j += 32) {
             const int e = sidx[tl * k + j];
+            if (!lmoe_check((unsigned)e < (unsigned)E, err)) {
+                sidx[tl * k + j] = -1;
+                continue;
+            }
             const int pos = mycur[e];
             mycur[e] = pos + 1;
             sidx[tl * k + j] = pos;  // slot, written out below
@@ -193,6 +200,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int pos = sidx[i];
         const size_t g = (size_t)t0 * k + i;
+        if (!lmoe_check((unsigned)pos < (unsigned)(T * k), err)) continue;
         slot[g] = pos;
         perm[pos] = t0 + i / k;
         wperm[pos] = w[g];
@@ -202,14 +210,16 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
 // dst[r, :] = src[perm[r], :] for r < *total (row_bytes multiple of 16). One
 // warp per row: the source row index is read once, and each lane keeps up to
 // eight 16-byte loads in flight before its stores.
-__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                const int* __restrict__ perm, const int* __restrict__ total,
-                                                int vec_per_row) {
+__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ src, int src_rows, int* err,
+                                                uint4* __restrict__ dst, const int* __restrict__ perm,
+                                                const int* __restrict__ total, int vec_per_row) {
     const int rows = *total;
     const int lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
-        const uint4* s = src + (long long)__ldg(perm + r) * vec_per_row;
+        const int pr = __ldg(perm + r);
+        if (!lmoe_check((unsigned)pr < (unsigned)src_rows, err)) continue;
+        const uint4* s = src + (long long)pr * vec_per_row;
         uint4* d = dst + (long long)r * vec_per_row;
         int c = lane;
         for (; c + 7 * 32 < vec_per_row; c += 8 * 32) {
@@ -226,13 +236,14 @@ __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ src, u
 // comb[t, :] = sum_{j ascending} o[slot[t, j], :]   (o already carries w)
 template <bool kBf16>
 __global__ void __launch_bounds__(256)
-    k_combine(const float4* __restrict__ o, const int* __restrict__ slot, void* __restrict__ comb, int T, int k,
-              int L4) {
+    k_combine(const float4* __restrict__ o, int o_rows, int* err, const int* __restrict__ slot, void* __restrict__ comb,
+              int T, int k, int L4) {
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         const int* sl = slot + (size_t)t * k;
         for (int c = threadIdx.x; c < L4; c += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < k; ++j) {
+                if (!lmoe_check((unsigned)sl[j] < (unsigned)o_rows, err)) continue;
                 float4 v = __ldg(&o[(size_t)sl[j] * L4 + c]);
                 acc.x += v.x;
                 acc.y += v.y;
@@ -363,7 +374,8 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
     const int E = h->cfg.num_experts, k = h->cfg.top_k;
     int* bc = reinterpret_cast<int*>(ws + p.blockcounts);
     const int32_t* idx = reinterpret_cast<const int32_t*>(ws + p.idx);
-    k_count<<<p.nblk, 256, E * sizeof(int), s>>>(idx, p.T, k, E, bc);
+    int* err = &reinterpret_cast<WsStats*>(ws + p.stats)->device_error;
+    k_count<<<p.nblk, 256, E * sizeof(int), s>>>(idx, p.T, k, E, bc, err);
     k_scan<<<1, 1024, 0, s>>>(bc, p.nblk, E, reinterpret_cast<int*>(ws + p.counts), counts_out,
                               reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.pfx128),
                               reinterpret_cast<int*>(ws + p.pfx64), reinterpret_cast<int*>(ws + p.pfxdec),
@@ -379,7 +391,7 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
                                                    reinterpret_cast<const int*>(ws + p.offsets),
                                                    reinterpret_cast<int*>(ws + p.perm),
                                                    reinterpret_cast<int*>(ws + p.slot),
-                                                   reinterpret_cast<float*>(ws + p.wperm));
+                                                   reinterpret_cast<float*>(ws + p.wperm), err);
     return cudaGetLastError();
 }
 
@@ -407,34 +419,35 @@ cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts,
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* src, void* dst, const int* perm, int rows_total_max, const int* total,
-                               int row_bytes, cudaStream_t s) {
+cudaError_t launch_gather_rows(const void* src, int src_rows, int* err, void* dst, const int* perm, int rows_total_max,
+                               const int* total, int row_bytes, int sms, cudaStream_t s) {
     const int vpr = row_bytes / 16;
-    int grid = grid_cap((long long)rows_total_max * 32, 256, 148 * 8);  // one warp per row
-    k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, total, vpr);
+    int grid = grid_cap((long long)rows_total_max * 32, 256, sms * 8);  // one warp per row
+    k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), src_rows, err, static_cast<uint4*>(dst), perm, total,
+                                  vpr);
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* o, const int* slot, void* comb, int T, int k, int L, bool out_bf16,
-                           cudaStream_t s) {
-    int grid = T < 148 * 8 ? T : 148 * 8;
+cudaError_t launch_combine(const float* o, int o_rows, int* err, const int* slot, void* comb, int T, int k, int L,
+                           bool out_bf16, int sms, cudaStream_t s) {
+    int grid = T < sms * 8 ? T : sms * 8;
     if (out_bf16)
-        k_combine<true><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), slot, comb, T, k, L / 4);
+        k_combine<true><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), o_rows, err, slot, comb, T, k, L / 4);
     else
-        k_combine<false><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), slot, comb, T, k, L / 4);
+        k_combine<false><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(o), o_rows, err, slot, comb, T, k, L / 4);
     return cudaGetLastError();
 }
 
-cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, cudaStream_t s) {
+cudaError_t launch_convert_x(const float* x, uint16_t* xb, long long n, int sms, cudaStream_t s) {
     long long n4 = n / 4;
-    k_convert<<<grid_cap(n4, 256, 148 * 16), 256, 0, s>>>(reinterpret_cast<const float4*>(x),
+    k_convert<<<grid_cap(n4, 256, sms * 16), 256, 0, s>>>(reinterpret_cast<const float4*>(x),
                                                           reinterpret_cast<uint2*>(xb), n4);
     return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out,
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* gamma, double eps, int T, int H, uint16_t* out, int sms,
                            cudaStream_t s) {
-    k_rmsnorm<<<T < 148 * 8 ? T : 148 * 8, 256, 0, s>>>(x, gamma, eps, T, H, out);
+    k_rmsnorm<<<T < sms * 8 ? T : sms * 8, 256, 0, s>>>(x, gamma, eps, T, H, out);
     return cudaGetLastError();
 }
 
@@ -444,10 +457,10 @@ cudaError_t launch_update_bias(const int32_t* counts, const float* bias_in, int 
     return cudaGetLastError();
 }
 
-cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n,
+cudaError_t launch_copy_routing(const int* idx, const float* w, int32_t* idx_out, float* w_out, long long n, int sms,
                                 cudaStream_t s) {
     if (!idx_out && !w_out) return cudaSuccess;
-    k_copy_routing<<<grid_cap(n, 256, 148 * 8), 256, 0, s>>>(idx, w, idx_out, w_out, n);
+    k_copy_routing<<<grid_cap(n, 256, sms * 8), 256, 0, s>>>(idx, w, idx_out, w_out, n);
     return cudaGetLastError();
 }
 

@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     k_select(const F* __restrict__ logits, const float* __restrict__ bias, int T, int E, int G, int Gk, int k,
              float scale, float delta, const int* __restrict__ list, const int* __restrict__ list_count,
              int32_t* __restrict__ idx, float* __restrict__ wgt, int* __restrict__ flaglist,
-             int* __restrict__ flag_count) {
+             int* __restrict__ flag_count, int* err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     F* c = reinterpret_cast<F*>(smem_raw) + (size_t)warp * 2 * E;
@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int n = list_count ? *list_count : T;
     for (int item = blockIdx.x * kWarps + warp; item < n; item += gridDim.x * kWarps) {
         const int t = list ? list[item] : item;
+        if (!lmoe_check((unsigned)t < (unsigned)T, err)) continue;
         const F* lg = logits + (size_t)t * E;
         for (int e = lane; e < E; e += 32) {
             F s = sigmoid_t(lg[e]);
@@ -234,7 +235,7 @@ constexpr int kEChunk = 64;
 template <bool kXf32>
 __global__ void __launch_bounds__(256)
     k_logits64(const void* __restrict__ x, const uint16_t* __restrict__ wr, int T, int E, int H,
-               const int* __restrict__ list, const int* __restrict__ list_count, double* __restrict__ out) {
+               const int* __restrict__ list, const int* __restrict__ list_count, double* __restrict__ out, int* err) {
     extern __shared__ __align__(16) double xrow[];
     const int n = list_count ? *list_count : T;
     const int chunks = (E + kEChunk - 1) / kEChunk;
@@ -243,6 +244,7 @@ __global__ void __launch_bounds__(256)
     for (long long item = blockIdx.x; item < (long long)n * chunks; item += gridDim.x) {
         const int li = (int)(item / chunks), ch = (int)(item % chunks);
         const int t = list ? list[li] : li;
+        if (!lmoe_check((unsigned)t < (unsigned)T, err)) continue;  // uniform over the block: no barrier skipped unevenly
         if (t != cur) {
             __syncthreads();
             for (int h = threadIdx.x; h < H; h += blockDim.x) {
@@ -305,7 +307,7 @@ cudaError_t launch_router_select(const lmoe_handle* h, const Plan& p, char* ws, 
     k_select<float, true><<<blocks, kWarps * 32, smem, s>>>(
         reinterpret_cast<const float*>(ws + p.logits), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
         c.routed_scaling_factor, h->flag_delta, nullptr, nullptr, reinterpret_cast<int32_t*>(ws + p.idx),
-        reinterpret_cast<float*>(ws + p.wgt), reinterpret_cast<int*>(ws + p.flaglist), &st->flagged);
+        reinterpret_cast<float*>(ws + p.wgt), reinterpret_cast<int*>(ws + p.flaglist), &st->flagged, &st->device_error);
     return cudaGetLastError();
 }
 
@@ -328,10 +330,10 @@ cudaError_t launch_router_logits64(const lmoe_handle* h, const void* x, const Pl
     }
     if (c.x_dtype == LMOE_FP32)
         k_logits64<true><<<blocks, 256, smem, s>>>(x, static_cast<const uint16_t*>(h->w.router_w), p.T,
-                                                   c.num_experts, c.hidden, list, cnt, out);
+                                                   c.num_experts, c.hidden, list, cnt, out, &st->device_error);
     else
         k_logits64<false><<<blocks, 256, smem, s>>>(x, static_cast<const uint16_t*>(h->w.router_w), p.T,
-                                                    c.num_experts, c.hidden, list, cnt, out);
+                                                    c.num_experts, c.hidden, list, cnt, out, &st->device_error);
     return cudaGetLastError();
 }
 
@@ -352,7 +354,7 @@ cudaError_t launch_router_select64(const lmoe_handle* h, const Plan& p, char* ws
         reinterpret_cast<const double*>(ws + p.logits64), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
         c.routed_scaling_factor, 0.f, all ? nullptr : reinterpret_cast<const int*>(ws + p.flaglist),
         all ? nullptr : &st->flagged, reinterpret_cast<int32_t*>(ws + p.idx), reinterpret_cast<float*>(ws + p.wgt),
-        nullptr, nullptr);
+        nullptr, nullptr, &st->device_error);
     return cudaGetLastError();
 }
 

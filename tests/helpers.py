@@ -6,17 +6,9 @@ import numpy as np
 import oracle
 import synth
 
-BF16_MAXABS = 2e-2      # stated bound (bf16 operands, fp32 accumulation)
+BF16_MAXABS = 2e-2      # stated bound (bf16 operands, fp32 accumulation), every GEMM path and width
 BF16_RELFRO = 1e-2
-FP32_RELFRO = 1e-5
-# Bound for the IEEE fp32 SIMT validation kernels at Nano/Ultra width only. Plain
-# fp32 accumulation flips ~0.02% of the bf16 roundings of z and of the expert
-# activations against an exactly rounding fp64 reference. A flipped z element
-# moves all k expert outputs of its token, and the output then moves by
-# 0.02-0.035 at the tail. The tensor-core paths re-round z exactly and meet the
-# stated 2e-2. The SIMT kernels do not re-round z, so they are held to this
-# derived bound; rel-Frobenius stays at the stated 1e-2.
-BF16_MAXABS_WIDE = 5e-2
+FP32_RELFRO = 1e-5      # stated bound of the fp32 validation mode
 
 
 def bf16_to_bits(t) -> np.ndarray:
@@ -81,14 +73,21 @@ def errors(y, ref):
     return float(np.abs(d).max()), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
 
 
-def assert_bf16_close(y, ref, wide=False):
+def assert_bf16_close(y, ref):
     ma, rf = errors(y, ref)
-    assert ma <= (BF16_MAXABS_WIDE if wide else BF16_MAXABS) and rf <= BF16_RELFRO, (ma, rf)
+    assert ma <= BF16_MAXABS and rf <= BF16_RELFRO, (ma, rf)
     return ma, rf
 
 
-def is_wide(shape):
-    return shape.H >= 4096
+def flagged_tokens(layer, T):
+    """Ids of the tokens whose routing the last call on the layer's workspace
+    re-decided in fp64 (the flag list the routing kernel writes)."""
+    import torch
+    n = layer.stats().flagged_tokens
+    if n == 0:
+        return np.zeros(0, dtype=np.int64)
+    lay = layer.layout(T)
+    return np.sort(layer.ws_view(lay.flag_list, (n,), torch.int32).cpu().numpy().astype(np.int64))
 
 
 def assert_fp32_close(y, ref):

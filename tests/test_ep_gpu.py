@@ -2,9 +2,11 @@
 
 - One rank (P = 1): the three stages give latentmoe_forward's y bit for bit,
   called directly and through ep_forward over a one-rank NCCL group.
-- Two ranks emulated in one process: two handles each holding half of the
+- Two and four ranks emulated in one process: handles each holding E/P of the
   experts, the all-to-all done with plain buffer copies (nothing waits across
-  ranks); each rank's y equals the single-handle forward of its tokens.
+  ranks); each rank's y equals the single-handle forward of its tokens bit for
+  bit, and the assembled y is within the stated tolerances of the fp64 oracle
+  (ragged and Nano shapes).
 """
 from dataclasses import replace
 
@@ -20,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE = 0, 1, 2
 RAGGED = LayerShape("ragged", T=333, H=512, L=256, E=64, k=6, G=4, Gk=2, I=384, Is=640)
+NANO_EP = synth.NANO_DECODE
 
 
 def stages(layer, x, n_src=1):
@@ -69,16 +72,19 @@ def test_one_rank_nvfp4_stages_equal_forward_bitwise():
     assert torch.equal(y, y_ref)
 
 
-def test_two_ranks_emulated_equal_single_handle():
+def emulate_ranks(shape, P, splits, dev=None):
+    """P expert-parallel ranks emulated in one process: P shard handles (experts
+    r*E/P .. (r+1)*E/P - 1 each), rank r on tokens splits[r]:splits[r+1] of x, the
+    all-to-all done as buffer copies (nothing waits across ranks). Returns the
+    ranks' y, the single-handle forward of the same tokens, and the inputs."""
     import torch
     import latentmoe_layer_b200 as lm
     from latentmoe_layer_b200 import ep
-    shape = RAGGED
-    P, El = 2, RAGGED.E // 2
-    dev = synth.device_inputs(shape, 0)
+    El = shape.E // P
+    dev = dev or synth.device_inputs(shape, 0)
     full = lm.LatentMoE(shape, dev, shape.T)
-    xs = [dev["x"][:170], dev["x"][170:]]
-    y_ref = [full.forward(x) for x in xs]
+    xs = [dev["x"][splits[r]:splits[r + 1]] for r in range(P)]
+    y_ref = [full.forward(x).clone() for x in xs]
     ranks = [lm.LatentMoE(shape, ep.shard_weights(dev, shape.E, r, P), shape.T, local_experts=El,
                           expert_base=r * El) for r in range(P)]
     fronts = [stages(ranks[r], xs[r]) for r in range(P)]
@@ -95,6 +101,7 @@ def test_two_ranks_emulated_equal_single_handle():
         o = torch.empty((rows.shape[0], shape.L), dtype=torch.float32, device="cuda")
         ranks[d].ep_experts(rows, w, rc, P, o)
         outs[d] = (o, [int(offs[s][d + 1] - offs[s][d]) for s in range(P)])
+    ys = []
     for r in range(P):
         back = []
         for d in range(P):
@@ -104,13 +111,42 @@ def test_two_ranks_emulated_equal_single_handle():
         send_o = torch.cat(back)
         y = torch.empty_like(y_ref[r])
         ranks[r].ep_back(send_o, y)
-        torch.cuda.synchronize()
-        ma = float((y - y_ref[r]).abs().max())
-        print("rank %d: max |y_ep - y| = %.3g, bitwise %s" % (r, ma, bool(torch.equal(y, y_ref[r]))))
-        assert ma <= 1e-4
-    # a shard handle refuses the single-GPU forward
-    with pytest.raises(lm.LmoeError):
-        ranks[0].forward(xs[0])
+        ys.append(y)
+    torch.cuda.synchronize()
+    for r in range(P):
+        assert ranks[r].stats().device_error == 0
+    return ys, y_ref, ranks, dev
+
+
+def check_ep_against_oracle(shape, P, splits):
+    """Each emulated rank's y equals the single-handle forward bit for bit (the experts
+    of a token are summed in ascending id on both paths), and the assembled y of all
+    tokens is within the stated tolerances of the fp64 oracle."""
+    import torch
+    ys, y_ref, ranks, dev = emulate_ranks(shape, P, splits)
+    for r in range(P):
+        assert torch.equal(ys[r], y_ref[r]), "rank %d differs from the single handle" % r
+    y = torch.cat(ys).cpu().numpy()
+    host = synth.host_inputs(shape)
+    yref, _, _ = H.oracle_forward(shape, host["x"][:splits[-1]], host)
+    ma, rf = H.assert_bf16_close(y, yref)
+    print("%s P=%d: bitwise equal to the single handle; vs oracle max_abs=%.3g rel_fro=%.3g" % (shape.name, P, ma, rf))
+    return ranks, dev
+
+
+def test_two_ranks_emulated_bitwise_and_oracle():
+    import latentmoe_layer_b200 as lm
+    ranks, dev = check_ep_against_oracle(RAGGED, 2, [0, 170, RAGGED.T])
+    with pytest.raises(lm.LmoeError):  # a shard handle refuses the single-GPU forward
+        ranks[0].forward(dev["x"][:170])
+
+
+def test_four_ranks_emulated_bitwise_and_oracle():
+    check_ep_against_oracle(RAGGED, 4, [0, 1, 120, 200, RAGGED.T])
+
+
+def test_two_ranks_emulated_nano_bitwise_and_oracle():
+    check_ep_against_oracle(NANO_EP, 2, [0, 61, NANO_EP.T])
 
 
 def test_ep_forward_one_rank_nccl_group():

@@ -113,7 +113,7 @@ def test_quantiser_bytes_match_oracle():
     assert float(g0[0]) == 1.0 and not c0.any() and not s0.any()
 
 
-def run_nvfp4(shape, path=GEMM_AUTO, wide=False):
+def run_nvfp4(shape, path=GEMM_AUTO):
     import torch
     layer, dev, q = nvfp4_layer(shape, path)
     T = shape.T
@@ -131,7 +131,7 @@ def run_nvfp4(shape, path=GEMM_AUTO, wide=False):
     assert np.array_equal(idx.cpu().numpy(), iref)
     assert np.array_equal(counts.cpu().numpy(), np.bincount(iref.ravel(), minlength=shape.E))
     np.testing.assert_allclose(w.cpu().numpy(), wref, rtol=2e-6, atol=1e-6)
-    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref, wide=wide)
+    ma, rf = H.assert_bf16_close(y.cpu().numpy(), yref)
     print("%s path=%d max_abs=%.3g rel_fro=%.3g" % (shape.name, path, ma, rf))
     return layer, dev, q, y
 
