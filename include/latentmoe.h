@@ -243,15 +243,24 @@ typedef enum {
                                     routing is exact whenever every fp32 choice score is within
                                     delta / 2 of its exact value                               */
     LMOE_OPT_SPIN_LIMIT = 3,     /* bound on device mbarrier polls before LMOE_ERR_TIMEOUT        */
-    LMOE_OPT_Z_RECHECK_DELTA = 4 /* margin of the exact re-rounding of z, in 1e-9 units (default
-                                    5000 = 5e-6; 0 disables). bf16 mode, tensor-core GEMMs: the
-                                    fc1 product is kept in fp32, rounded to bf16 nearest-even,
-                                    and every element whose fp32 value lies within the margin of
-                                    a bf16 rounding midpoint is recomputed as an fp64 sum of the
-                                    exact bf16 products and rounded again, so z is the exactly
-                                    rounded x W_fc1^T whenever the fp32 error is below the margin
-                                    (z is the rounding point that every routed expert of a token
-                                    reads). Valid range 0 .. 1e8. */
+    LMOE_OPT_Z_RECHECK_DELTA = 4,/* margin scale d of the exact re-rounding of z, in 1e-9 units
+                                    (default 6000 = 6e-6; 0 disables). bf16 mode: the fc1
+                                    product is kept in fp32, rounded to bf16 nearest-even, and
+                                    every element whose fp32 value lies within d (1 + 0.4 |z|) of
+                                    a bf16 rounding midpoint is recomputed as an error-free sum
+                                    of the exact bf16 products and rounded again, so z is the
+                                    exactly rounded x W_fc1^T whenever the fp32 error of each
+                                    element is below its margin (z is the rounding point that
+                                    every routed expert of a token reads). Valid 0 .. 1e8. */
+    LMOE_OPT_ACT_RECHECK_TAU = 5 /* threshold tau of the exact re-rounding of the relu2
+                                    activations (expert and shared-expert up projections), in
+                                    1e-3 units (default 2000 = 2.0; 0 disables). bf16 mode,
+                                    bf16 experts: an activation a = max(h, 0)^2 with h > tau whose
+                                    fp32 value lies within the fp32 accumulation error of h
+                                    (1.6e-6 + 0.9e-6 h, carried through the square) of a bf16
+                                    rounding midpoint is recomputed exactly. A flipped rounding
+                                    moves the output by about one bf16 step of a, which grows as
+                                    h^2, so the large activations carry most of that error. */
 } lmoe_option;
 lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long value);
 
@@ -265,6 +274,11 @@ typedef struct {
                                failed (a call that returned LMOE_ERR_CUDA), 0 if none     */
     int z_rechecked;        /* z elements listed and re-rounded exactly (LMOE_OPT_Z_RECHECK_DELTA);
                                the list has room for all T*L elements                    */
+    int ae_rechecked;       /* expert activations listed for exact re-rounding
+                               (LMOE_OPT_ACT_RECHECK_TAU); the list holds max(T*Is,
+                               T*top_k*expert_inter)/256 + 64 entries, and elements past
+                               it keep their fp32-decided rounding                      */
+    int as_rechecked;       /* shared-expert activations listed, same list room          */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;
  * for tests and benchmarks, not for the hot path). */

@@ -26,7 +26,7 @@ LMOE_OK, LMOE_ERR_INVALID_ARG, LMOE_ERR_UNSUPPORTED, LMOE_ERR_WORKSPACE, LMOE_ER
 LMOE_BF16, LMOE_FP32 = 0, 1
 LMOE_MODE_BF16, LMOE_MODE_FP32 = 0, 1
 LMOE_EXPERTS_BF16, LMOE_EXPERTS_NVFP4 = 0, 1
-OPT_GEMM_PATH, OPT_ROUTER_FP64_ALL, OPT_FLAG_DELTA, OPT_SPIN_LIMIT, OPT_Z_RECHECK_DELTA = range(5)
+OPT_GEMM_PATH, OPT_ROUTER_FP64_ALL, OPT_FLAG_DELTA, OPT_SPIN_LIMIT, OPT_Z_RECHECK_DELTA, OPT_ACT_RECHECK_TAU = range(6)
 GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 
 EXPORTS = ["latentmoe_create", "latentmoe_workspace_size", "latentmoe_route", "latentmoe_forward",
@@ -53,7 +53,8 @@ class lmoe_weights(ctypes.Structure):
 class lmoe_stats(ctypes.Structure):
     _fields_ = [("flagged_tokens", ctypes.c_int), ("distinct_experts", ctypes.c_int),
                 ("max_expert_tokens", ctypes.c_int), ("device_error", ctypes.c_int),
-                ("kernel_launches", ctypes.c_int), ("cuda_error", ctypes.c_int), ("z_rechecked", ctypes.c_int)]
+                ("kernel_launches", ctypes.c_int), ("cuda_error", ctypes.c_int), ("z_rechecked", ctypes.c_int),
+                ("ae_rechecked", ctypes.c_int), ("as_rechecked", ctypes.c_int)]
 
 
 class lmoe_ws_layout(ctypes.Structure):

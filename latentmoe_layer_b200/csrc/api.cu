@@ -116,6 +116,11 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     // shares the expert activation buffer (free until the expert up GEMM) when that
     // is large enough (top_k * I >= 4 L), else it has its own
     p.zlist = (A * I * act >= (size_t)T * L * 8) ? p.aperm : take((size_t)T * L * 8);
+    // activation re-rounding list (the shared expert's, then the experts': one at a time), room
+    // for 1/256 of the larger activation set, far above the ~1e-4 that the margins list
+    p.alist_cap = (int)std::min<size_t>(std::max((size_t)T * Is, A * I) / 256 + 64, 0x7FFFFFFF);
+    p.alist = take((size_t)p.alist_cap * 8);
+    p.zrowtab = take((size_t)T * ((L + 2047) / 2048) * 16);  // one {row, first, entries} per 2048-column segment
     p.total = off;
     return true;
 }
@@ -183,6 +188,9 @@ struct Ctx {
     cudaStream_t s;
     DeviceRouting r;
     int* err;
+    WsStats* st;          // the call's statistics block
+    int2* alist;          // activation re-rounding list and its room
+    int alist_cap;
     bool decode;  // swap-AB tiles for the expert GEMMs and the dense GEMMs
     bool simt;
 };
@@ -241,6 +249,19 @@ cudaError_t run_gemm_nvfp4(Ctx& c, GemmProblem* pr, const Operand& act) {
     pr->a_map[0] = 0;
     pr->b_map[0] = -1;
     return launch_gemm_tc_nvfp4(&map, 1, pr, 1, bn, c.r, c.err, c.h->spin_limit, c.s);
+}
+
+// The exact re-rounding list of a relu2 activation problem (see rr_flag).
+void set_act_recheck(const Ctx& c, GemmProblem& pr, int* count) {
+    const double tau = c.h->act_tau, c0 = c.h->act_c0, c1 = c.h->act_c1;
+    pr.rr_list = c.alist;
+    pr.rr_count = count;
+    pr.rr_cap = c.alist_cap;
+    const float tau2 = (float)(tau * tau);
+    memcpy(&pr.rr_tau2_bits, &tau2, 4);
+    // margin of a = h^2 over an fp32 ulp of a (>= a 2^-24), at its largest (a = tau^2)
+    pr.rr_ulps = (uint32_t)ceil(16777216.0 * (c0 / (tau * tau) + c0 + 2.0 * c1));
+    if (pr.rr_ulps > 0x4000u) pr.rr_ulps = 0x4000u;
 }
 
 GemmProblem make_problem(int grouped, int m_rows, int n, int epi, void* out, long long ldo) {
@@ -352,6 +373,9 @@ Ctx make_ctx(lmoe_handle* h, const Plan& p, void* ws, void* stream) {
     c.r.rec256 = reinterpret_cast<const int4*>(c.ws + p.rec256);
     c.r.E = h->cfg.num_experts;
     c.err = &reinterpret_cast<WsStats*>(c.ws + p.stats)->device_error;
+    c.st = reinterpret_cast<WsStats*>(c.ws + p.stats);
+    c.alist = reinterpret_cast<int2*>(c.ws + p.alist);
+    c.alist_cap = p.alist_cap;
     const lmoe_config& cf = h->cfg;
     c.simt = h->gemm_path == 3 || cf.mode == LMOE_MODE_FP32;
     if (h->gemm_path == 1 || h->gemm_path == 4) c.decode = false;
@@ -393,12 +417,16 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         xa = ws_c + p.xbf;
         xa_f32 = false;
     }
+    const bool act_rr = bf16 && h->act_tau > 0.f;
     {
         GemmProblem pr[2] = {make_problem(0, p.T, L, bf16 && !zcheck ? EPI_BF16 : EPI_F32, ws_c + (zcheck ? p.o : p.z),
                                           L),
                              make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is)};
         pr[0].kdim[0] = H;
         pr[1].kdim[0] = H;
+        // fc1 in chunks of 4 k-blocks when z is re-rounded: half the fp32 error, half the list
+        if (zcheck) pr[0].chunk_kb = 4;
+        if (act_rr) set_act_recheck(c, pr[1], &c.st->asflagged);
         pr[0].a_ptr[0] = xa;
         pr[0].b_ptr[0] = h->w.fc1_w;
         pr[1].a_ptr[0] = xa;
@@ -410,13 +438,21 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
     if (zcheck) {
         const int cap = (int)std::min<long long>((long long)p.T * L, 0x7FFFFFFF);  // T * L < 2^31 (create)
         int2* list = reinterpret_cast<int2*>(ws_c + p.zlist);
-        int* count = &reinterpret_cast<WsStats*>(ws_c + p.stats)->zflagged;
+        int* count = &c.st->zflagged;
         uint16_t* z = reinterpret_cast<uint16_t*>(ws_c + p.z);
+        int4* rowtab = reinterpret_cast<int4*>(ws_c + p.zrowtab);
         LMOE_LAUNCH(1, launch_z_round_flag(reinterpret_cast<const float*>(ws_c + p.o), z, p.T, L, h->zcheck_delta,
-                                           list, cap, count, h->num_sms, c.s));
-        LMOE_LAUNCH(1, launch_z_recheck(static_cast<const uint16_t*>(xa), static_cast<const uint16_t*>(h->w.fc1_w),
-                                        H, p.T, c.err, list, count, cap, z, L, h->num_sms, c.s));
+                                           0.4f * h->zcheck_delta, list, cap, count, rowtab, &c.st->zrows, h->num_sms,
+                                           c.s));
+        LMOE_LAUNCH(1, launch_recheck_rows(static_cast<const uint16_t*>(xa), p.T,
+                                           static_cast<const uint16_t*>(h->w.fc1_w), L, H, c.err, list, cap, rowtab,
+                                           &c.st->zrows, z, L, h->num_sms, c.s));
     }
+    if (act_rr)
+        LMOE_LAUNCH(1, launch_recheck(true, static_cast<const uint16_t*>(xa), p.T,
+                                      static_cast<const uint16_t*>(h->w.shared_up_w), Is, H, c.err, c.alist,
+                                      &c.st->asflagged, c.alist_cap, reinterpret_cast<uint16_t*>(ws_c + p.as), Is,
+                                      h->num_sms, c.s));
     mark(c, 2);
     LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, p.T, c.err, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
                                       reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, h->num_sms, c.s));
@@ -434,11 +470,13 @@ lmoe_status stage_experts(Ctx& c, const void* rows, long long n, const float* ro
     const bool bf16 = cf.mode == LMOE_MODE_BF16;
     const bool fp4 = cf.expert_format == LMOE_EXPERTS_NVFP4;
     const int L = cf.latent, I = cf.expert_inter, Ew = experts_held(cf);
+    const bool act_rr = bf16 && !fp4 && h->act_tau > 0.f;
     {
         GemmProblem pr = make_problem(1, 0, I, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, a_buf, I);
         pr.kdim[0] = L;
         pr.b_rows_per_expert = I;
         pr.expert_mod = expert_mod;
+        if (act_rr) set_act_recheck(c, pr, &c.st->aeflagged);
         pr.a_ptr[0] = rows;
         pr.b_ptr[0] = h->w.up_w;
         Operand a[1][2] = {{{rows, n}, {nullptr, 0}}};
@@ -452,6 +490,11 @@ lmoe_status stage_experts(Ctx& c, const void* rows, long long n, const float* ro
             LMOE_LAUNCH(1, run_gemm(c, &pr, 1, a, b, !bf16));
         }
     }
+    if (act_rr)
+        LMOE_LAUNCH(1, launch_recheck(true, static_cast<const uint16_t*>(rows), (int)n,
+                                      static_cast<const uint16_t*>(h->w.up_w), Ew * I, L, c.err, c.alist,
+                                      &c.st->aeflagged, c.alist_cap, static_cast<uint16_t*>(a_buf), I, h->num_sms,
+                                      c.s));
     mark(c, 4);
     {
         GemmProblem pr = make_problem(1, 0, L, EPI_SCALE_F32, o, L);
@@ -536,7 +579,8 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
 // Workspace of latentmoe_ep_experts: the scan of the received blocks and the
 // expert activations of the received rows.
 struct EpPlan {
-    size_t total, stats, bcounts, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64, rec128, rec256, a;
+    size_t total, stats, bcounts, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64, rec128, rec256, a, alist;
+    int alist_cap;
 };
 
 void ep_plan_of(const lmoe_config& c, int n_rows, int nb, EpPlan& p) {
@@ -560,6 +604,8 @@ void ep_plan_of(const lmoe_config& c, int n_rows, int nb, EpPlan& p) {
     p.rec128 = take((n / 128 + nb) * 16);
     p.rec256 = take((n / 256 + nb) * 16);
     p.a = take(n * c.expert_inter * (c.mode == LMOE_MODE_BF16 ? 2 : 4));
+    p.alist_cap = (int)std::min<size_t>(n * c.expert_inter / 256 + 64, 0x7FFFFFFF);
+    p.alist = take((size_t)p.alist_cap * 8);
     p.total = off;
 }
 
@@ -701,6 +747,10 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
             if (v < 1 || v > 0xFFFFFFFFLL) return LMOE_ERR_INVALID_ARG;
             h->spin_limit = (unsigned)v;
             return LMOE_OK;
+        case LMOE_OPT_ACT_RECHECK_TAU:
+            if (v < 0 || v > 1000000) return LMOE_ERR_INVALID_ARG;
+            h->act_tau = (float)(v * 1e-3);
+            return LMOE_OK;
     }
     return LMOE_ERR_INVALID_ARG;
 }
@@ -730,6 +780,8 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
     out->kernel_launches = h->launches;
     out->cuda_error = h->last_cuda_error;
     out->z_rechecked = st.zflagged;
+    out->ae_rechecked = st.aeflagged;
+    out->as_rechecked = st.asflagged;
     return LMOE_OK;
 }
 
@@ -812,6 +864,9 @@ lmoe_status latentmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const fl
     c.r.rec256 = reinterpret_cast<const int4*>(c.ws + q.rec256);
     c.r.E = nb;
     c.err = &reinterpret_cast<WsStats*>(c.ws + q.stats)->device_error;
+    c.st = reinterpret_cast<WsStats*>(c.ws + q.stats);
+    c.alist = reinterpret_cast<int2*>(c.ws + q.alist);
+    c.alist_cap = q.alist_cap;
     c.simt = h->gemm_path == 3 || cf.mode == LMOE_MODE_FP32;
     if (h->gemm_path == 1 || h->gemm_path == 4) c.decode = false;
     else if (h->gemm_path == 2) c.decode = true;

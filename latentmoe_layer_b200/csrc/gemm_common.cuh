@@ -47,6 +47,36 @@ struct TileInfo {
     bool half;   // non-swapped tile with <= 64 valid rows: M = 64 MMAs (the expert's ragged tail)
 };
 
+// Appends the elements this thread marked in mask (bit i of word w = its
+// accumulator column c0 + 32 w + i), n of them, to the problem's re-rounding
+// list with one atomic per warp: an inclusive scan of the lanes' counts gives
+// each lane its run of entries. Called by all 32 lanes of the warp.
+template <int kW>
+__device__ __forceinline__ void rr_append_warp(const GemmProblem& pr, int n, const uint32_t (&mask)[kW],
+                                               const TileInfo& ti, int lane_row, int c0, bool swap) {
+    const int lane = threadIdx.x & 31;
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    int base = 0;
+    if (lane == 31) base = atomicAdd(pr.rr_count, total);
+    int pos = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - n;
+    for (int w = 0; w < kW; ++w) {
+        uint32_t m = mask[w];
+        while (m) {
+            const int i = w * 32 + __ffs(m) - 1;
+            m &= m - 1u;
+            const int r = swap ? c0 + i : lane_row, col = swap ? lane_row : c0 + i;
+            if (pos < pr.rr_cap) pr.rr_list[pos] = make_int2(ti.row0 + r, ti.wrow0 + col);
+            ++pos;
+        }
+    }
+}
+
 template <int BN, bool kSwap>
 struct Shape {
     static constexpr int XR = 128;            // rows of the MMA A operand tile
@@ -184,6 +214,25 @@ __device__ __forceinline__ void epilogue_store(const GemmProblem& pr, const Tile
         for (int i = 0; i < CW; ++i) {
             float a = fmaxf(acc[i], 0.f);
             acc[i] = a * a;
+        }
+        // exact re-rounding list (bf16 mode): large activations near a rounding midpoint, marked
+        // in a bit mask first, then listed (a few per tile) with one atomic per warp. All 32
+        // lanes of the warp are here.
+        if (epi == EPI_RELU2_BF16 && pr.rr_list != nullptr) {
+            constexpr int kW = (CW + 31) / 32;
+            uint32_t mask[kW];
+#pragma unroll
+            for (int w = 0; w < kW; ++w) mask[w] = 0u;
+#pragma unroll
+            for (int i = 0; i < CW; ++i) {
+                // non-swapped: row lane_row of the tile, weight row c0 + i; swapped: the reverse
+                const int r = kSwap ? c0 + i : lane_row;
+                if (r < ti.rows && rr_flag(acc[i], pr.rr_tau2_bits, pr.rr_ulps)) mask[i >> 5] |= 1u << (i & 31);
+            }
+            int n = 0;
+#pragma unroll
+            for (int w = 0; w < kW; ++w) n += __popc(mask[w]);
+            if (__any_sync(0xFFFFFFFFu, n != 0)) rr_append_warp<kW>(pr, n, mask, ti, lane_row, c0, kSwap);
         }
     }
     if (!kSwap && pr.resid && lane_row < ti.rows) {  // block residual: out = resid + acc (fp32)

@@ -90,6 +90,9 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const GemmProblem pr, const D
             if (pr.epi == EPI_RELU2_BF16 || pr.epi == EPI_RELU2_F32) {
                 v = fmaxf(v, 0.f);
                 v = v * v;
+                // exact re-rounding list (bf16 mode): large activations near a rounding midpoint
+                if (pr.epi == EPI_RELU2_BF16 && pr.rr_list && rr_flag(v, pr.rr_tau2_bits, pr.rr_ulps))
+                    rr_append(pr, (int)row, wrow0 + tx * 4 + j);
             }
             if (pr.epi == EPI_SCALE_F32) v *= pr.row_scale[row];
             const long long o = row * pr.ldo + col0 + tx * 4 + j;

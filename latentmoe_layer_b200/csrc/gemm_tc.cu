@@ -131,9 +131,10 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
             const int kb_total = tile_kblocks(P.prob[ti.p]);
+            const int ck = P.prob[ti.p].chunk_kb ? P.prob[ti.p].chunk_kb : CK;
             // M = 64 puts D rows 16q..16q+15 in TMEM lanes 32q..32q+15 (q = lane quarter)
             const uint32_t idesc = ti.half ? idesc_half : idesc_full;
-            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += CK) {
+            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += ck) {
                 // next chunk accumulator must have been drained by the epilogue
                 if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, P.spin, err)) {
                     ok = false;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * BN);
-                const int kb1 = min(kb_total, kb0 + CK);
+                const int kb1 = min(kb_total, kb0 + ck);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
                         ok = false;
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
             const GemmProblem& pr = P.prob[ti.p];
             const int kb_total = tile_kblocks(pr);
+            const int ck = pr.chunk_kb ? pr.chunk_kb : CK;
 #if LMOE_PROMOTE_F64
             double accd[CW];
 #pragma unroll
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
 #pragma unroll
             for (int i = 0; i < CW; ++i) acc[i] = 0.f;
 #endif
-            for (int kb0 = 0; kb0 < kb_total; kb0 += CK) {
+            for (int kb0 = 0; kb0 < kb_total; kb0 += ck) {
                 if (!mbar_wait_bounded(&cfull[buf], bphase, P.spin, err)) {
                     ok = false;
                     break;

@@ -10,7 +10,15 @@ struct lmoe_handle {
     int gemm_path = 0;         // lmoe_option LMOE_OPT_GEMM_PATH
     int fp64_all = 0;          // LMOE_OPT_ROUTER_FP64_ALL
     float flag_delta = 2e-5f;  // LMOE_OPT_FLAG_DELTA (10x the largest fp32 score error seen at Ultra width, x2)
-    float zcheck_delta = 5e-6f;  // LMOE_OPT_Z_RECHECK_DELTA (mean |fp32 - exact| of z: ~3e-7)
+    // LMOE_OPT_Z_RECHECK_DELTA: margin of z's exact re-rounding, zcheck_delta * (1 + 0.4 |z|);
+    // >= 4x the largest fp32 error of z measured at Ultra width with fc1 in chunks of 4 k-blocks
+    // (1.16e-6 + 0.45e-6 |z| over 524288 elements; the smallest ratio seen is 4.5)
+    float zcheck_delta = 6e-6f;
+    // LMOE_OPT_ACT_RECHECK_TAU: relu2 activations with h above this are re-rounded exactly when
+    // within the accumulation-error margin (act_c0 + act_c1 h: the largest fp32 error measured at
+    // K = 8192 in chunks of 8 k-blocks) of a bf16 midpoint
+    float act_tau = 2.0f;
+    float act_c0 = 1.6e-6f, act_c1 = 0.9e-6f;
     unsigned spin_limit = 1u << 24;
     int num_sms = 148;
     int launches = 0;                  // kernels launched by the last call

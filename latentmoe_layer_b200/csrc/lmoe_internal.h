@@ -42,7 +42,10 @@ struct WsStats {
     int max_count;      // largest per-expert count
     int device_error;   // lmoe_status from a device check
     int zflagged;       // z elements listed for the exact re-rounding
-    int pad[59];
+    int aeflagged;      // expert activations listed for the exact re-rounding
+    int asflagged;      // shared-expert activations listed for the exact re-rounding
+    int zrows;          // row segments of z with listed elements (entries of the row table)
+    int pad[56];
 };
 
 // Epilogue kinds of the GEMM kernels.
@@ -84,7 +87,37 @@ struct GemmProblem {
     // g % expert_mod (expert parallelism: groups are (source rank, local expert)
     // blocks of received rows in arrival order).
     int expert_mod;
+    // K accumulated per TMEM chunk, in k-blocks (0: the engine's default).
+    int chunk_kb;
+    // Exact re-rounding list of a relu2 bf16 output (rr_list non-null): every
+    // activation a = max(h, 0)^2 above rr_tau2_bits (the fp32 pattern of tau^2)
+    // whose fp32 value lies within rr_ulps fp32 ulps of a bf16 rounding midpoint
+    // is appended as (row, weight row) for an exact recomputation (rr_flag).
+    int2* rr_list;
+    int* rr_count;
+    int rr_cap;
+    uint32_t rr_tau2_bits, rr_ulps;
 };
+
+// Whether a = max(h, 0)^2, computed in fp32, is above tau^2 and within `ulps`
+// fp32 ulps of a bf16 rounding midpoint. For a positive fp32 value the bf16
+// values are the patterns with zero low 16 bits and the only midpoint between
+// two of them has low bits 0x8000, so the distance in ulps is |low16 - 0x8000|.
+// The host derives `ulps` from the accumulation-error margin of h (c0 + c1 h,
+// carried through the square: about 2h (c0 + c1 h) <= c0 + (c0 + 2 c1) a, with
+// h <= (a + 1) / 2) and from ulp(a) >= a 2^-24, so the test lists every
+// element the margin asks for and at most a few times more.
+__device__ __forceinline__ bool rr_flag(float a, uint32_t tau2_bits, uint32_t ulps) {
+    const uint32_t u = __float_as_uint(a);
+    return u > tau2_bits && (u & 0xFFFFu) - (0x8000u - ulps) < 2u * ulps;
+}
+
+// Lists one element for re-rounding (rare: a handful per tile). Entries past the
+// list's room are counted, not written.
+static __device__ __noinline__ void rr_append(const GemmProblem& pr, int row, int wrow) {
+    const int pos = atomicAdd(pr.rr_count, 1);
+    if (pos < pr.rr_cap) pr.rr_list[pos] = make_int2(row, wrow);
+}
 
 struct DeviceRouting {
     const int* offsets;     // [E+1] permuted row offset of each expert
@@ -106,7 +139,8 @@ struct DeviceRouting {
 struct Plan {
     size_t total;
     size_t stats, logits, logits64, flaglist, idx, wgt, counts, offsets, pfx128, pfx64, pfxdec, pfx256, rec32, rec64,
-        rec128, rec256, blockcounts, perm, slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as, zlist;
+        rec128, rec256, blockcounts, perm, slot, wperm, xbf, xnorm, z, zperm, aperm, o, comb, as, zlist, alist, zrowtab;
+    int alist_cap;  // entries of the activation re-rounding list
     int T, A, nblk;
 };
 
@@ -124,11 +158,13 @@ cudaError_t launch_permute(const lmoe_handle* h, const Plan& p, char* ws, int32_
 cudaError_t launch_group_scan(int* blockcounts, int nb, int n_rows, int* counts, int* offsets, int* pfx128, int* pfx64,
                               int* pfxdec, int* pfx256, int4* rec32, int4* rec64, int4* rec128, int4* rec256,
                               WsStats* st, cudaStream_t s);
-cudaError_t launch_z_round_flag(const float* z32, uint16_t* z, int rows, int L, float delta, int2* list, int cap,
-                                int* count, int sms, cudaStream_t s);
-cudaError_t launch_z_recheck(const uint16_t* x, const uint16_t* w, int K, int rows, int* err, const int2* list,
-                             const int* count, int cap,
-                             uint16_t* z, int L, int sms, cudaStream_t s);
+cudaError_t launch_z_round_flag(const float* z32, uint16_t* z, int rows, int L, float m0, float m1, int2* list, int cap,
+                                int* count, int4* rowtab, int* nrowtab, int sms, cudaStream_t s);
+cudaError_t launch_recheck_rows(const uint16_t* A, int a_rows, const uint16_t* W, int w_rows, int K, int* err,
+                                const int2* list, int cap, const int4* rowtab, const int* nrowtab, uint16_t* out,
+                                int ldo, int sms, cudaStream_t s);
+cudaError_t launch_recheck(bool relu2, const uint16_t* A, int a_rows, const uint16_t* W, int w_rows, int K, int* err,
+                           const int2* list, const int* count, int cap, uint16_t* out, int ldo, int sms, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, int src_rows, int* err, void* dst, const int* perm, int rows_total_max,
                                const int* offsets_E,
                                int row_bytes, int sms, cudaStream_t s);

@@ -171,7 +171,8 @@ def test_call_errors_leave_outputs_untouched(lib):
     assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, -1) == lm.LMOE_ERR_INVALID_ARG
     assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 100000001) == lm.LMOE_ERR_INVALID_ARG
     assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 0) == lm.LMOE_OK
-    assert lm.latentmoe_set_option(layer.h, 5, 0) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_ACT_RECHECK_TAU, -1) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, 6, 0) == lm.LMOE_ERR_INVALID_ARG
 
 
 @pytest.mark.gpu
@@ -223,4 +224,4 @@ def test_binding_matches_header_stats_and_options():
     opts = dict((k, int(v)) for k, v in re.findall(r"LMOE_OPT_(\w+)\s*=\s*(\d+)", hdr))
     assert opts == {"GEMM_PATH": lm.OPT_GEMM_PATH, "ROUTER_FP64_ALL": lm.OPT_ROUTER_FP64_ALL,
                     "FLAG_DELTA": lm.OPT_FLAG_DELTA, "SPIN_LIMIT": lm.OPT_SPIN_LIMIT,
-                    "Z_RECHECK_DELTA": lm.OPT_Z_RECHECK_DELTA}
+                    "Z_RECHECK_DELTA": lm.OPT_Z_RECHECK_DELTA, "ACT_RECHECK_TAU": lm.OPT_ACT_RECHECK_TAU}

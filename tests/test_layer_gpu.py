@@ -92,6 +92,7 @@ def test_exact_z_rounding_meets_the_stated_tolerance_at_full_width():
     """Nano over all its rows. With z re-rounded exactly (the default) y is within the stated max-abs 2e-2;
     a margin 8x wider gives the same y bit for bit (no fp32 error escapes the default margin on these
     inputs); margin 0 turns the re-rounding off and the error returns to the fp32 floor."""
+    DEFAULT, WIDE = 6000, 48000
     import torch
     shape = NANO_DECODE
     layer, dev = H.device_layer(shape)
@@ -102,7 +103,7 @@ def test_exact_z_rounding_meets_the_stated_tolerance_at_full_width():
     n_default = layer.stats().z_rechecked
     d = y.cpu().numpy().astype(np.float64) - yref
     ma, rf = float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(yref))
-    layer.set_option(lm_opt("OPT_Z_RECHECK_DELTA"), 40000)
+    layer.set_option(lm_opt("OPT_Z_RECHECK_DELTA"), WIDE)
     y8 = layer.forward(dev["x"]).clone()
     torch.cuda.synchronize()
     n_wide = layer.stats().z_rechecked
@@ -113,7 +114,7 @@ def test_exact_z_rounding_meets_the_stated_tolerance_at_full_width():
     d0 = y0.cpu().numpy().astype(np.float64) - yref
     print("nano exact z: rechecked %d of %d (x8 margin: %d), max_abs=%.3g rel_fro=%.3g; without: max_abs=%.3g" %
           (n_default, shape.T * shape.L, n_wide, ma, rf, float(np.abs(d0).max())))
-    assert 0 < n_default < n_wide < shape.T * shape.L // 4
+    assert 0 < n_default < n_wide < shape.T * shape.L // 2
     assert torch.equal(y, y8)
     assert ma <= 2e-2 and rf <= 1e-2
 
@@ -166,8 +167,9 @@ def _full_size_parity(shape, n_rows, seed, path=GEMM_AUTO):
     ma, rf = H.assert_bf16_close(y.cpu().numpy()[rows], yref)
     hot = float(gc[:16].sum()) / gc.sum()
     print("%s path=%d rows=%d max_abs=%.3g rel_fro=%.3g flagged=%d (all in the sample) distinct=%d max_count=%d "
-          "hot16_share=%.3f" % (shape.name, path, len(rows), ma, rf, st.flagged_tokens, st.distinct_experts,
-                                st.max_expert_tokens, hot))
+          "hot16_share=%.3f re-rounded: z %d, a_e %d, a_s %d" %
+          (shape.name, path, len(rows), ma, rf, st.flagged_tokens, st.distinct_experts, st.max_expert_tokens, hot,
+           st.z_rechecked, st.ae_rechecked, st.as_rechecked))
     return layer
 
 
@@ -265,7 +267,7 @@ def test_nano_fp32_validation_mode_full():
 
 # ---------------------------------------------------------------- margins of the exactness re-checks
 DEFAULT_FLAG_DELTA = 2e-5   # LMOE_OPT_FLAG_DELTA default (include/latentmoe.h)
-DEFAULT_Z_DELTA = 5e-6      # LMOE_OPT_Z_RECHECK_DELTA default
+DEFAULT_Z_DELTA = 6e-6      # LMOE_OPT_Z_RECHECK_DELTA default: the margin is d (1 + 0.4 |z|)
 FP32_EVAL_BUDGET = 4 * 2.0 ** -24  # fp32 sigmoid (expf, add, divide) and bias add of a score below 1.2
 
 
@@ -295,9 +297,11 @@ def test_router_fp32_error_is_far_inside_the_flag_margin():
 
 def test_z_fp32_error_is_far_inside_the_rerounding_margin():
     """z = bf16(x W_fc1^T) is re-rounded exactly for every element whose fp32 value lies within
-    the margin of a bf16 rounding midpoint: that is exact when the fp32 error is below the margin.
-    On 256 rows of the 16384-token Ultra batch, the largest |fp32 z - exact z| must leave a 10x
-    margin, and the stored z must equal the exact rounding bit for bit."""
+    the margin d (1 + 0.4 |z|) of a bf16 rounding midpoint: that is exact when each element's fp32
+    error is below its margin. On 256 rows of the 16384-token Ultra batch every element's
+    |fp32 z - exact z| must leave a 4x margin (a 10x margin would list ~2.5x more elements, each
+    re-computed from 32 KB of operand rows), and the stored z must equal the exact rounding bit
+    for bit."""
     import torch
     shape = ULTRA_PREFILL
     layer, dev = H.device_layer(shape)
@@ -325,9 +329,10 @@ def test_z_fp32_error_is_far_inside_the_rerounding_margin():
                   (lo, hi, int(m.sum()), float(d[m].max()), float((d[m] / np.maximum(az[m], 1e-30)).max())))
     ref = np.vectorize(oracle.round_bf16)(exact).astype(np.float32).view(np.uint32) >> 16
     flips = int((zb != ref.astype(np.uint16)).sum())
-    print("z: max |fp32 - exact| %.3g; margin %.3g (%.0fx); rechecked %d of %d; elements != exact rounding: %d" %
-          (err, DEFAULT_Z_DELTA, DEFAULT_Z_DELTA / err, layer.stats().z_rechecked, T * L, flips))
-    assert DEFAULT_Z_DELTA >= 10 * err
+    ratio = float((DEFAULT_Z_DELTA * (1 + 0.4 * az) / np.maximum(d, 1e-30)).min())
+    print("z: max |fp32 - exact| %.3g; smallest margin / error over all elements %.1fx; rechecked %d of %d; "
+          "elements != exact rounding: %d" % (err, ratio, layer.stats().z_rechecked, T * L, flips))
+    assert ratio >= 4
     assert flips == 0
 
 
