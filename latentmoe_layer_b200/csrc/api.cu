@@ -251,6 +251,22 @@ cudaError_t run_gemm_nvfp4(Ctx& c, GemmProblem* pr, const Operand& act) {
     return launch_gemm_tc_nvfp4(&map, 1, pr, 1, bn, c.r, c.err, c.h->spin_limit, c.s);
 }
 
+// TMEM accumulation chunks (k-blocks of 64) per GEMM: a chunk bounds the size of
+// the partial sums the tensor core accumulates, which matters where the output
+// is rounded to bf16; fp32 outputs (expert down, output GEMM) take K whole.
+#ifndef LMOE_CHUNK_UP
+#define LMOE_CHUNK_UP 0      // expert up (a_e, re-rounded): the engine's default
+#endif
+#ifndef LMOE_CHUNK_DOWN
+#define LMOE_CHUNK_DOWN 0
+#endif
+#ifndef LMOE_CHUNK_OUT
+#define LMOE_CHUNK_OUT 0
+#endif
+#ifndef LMOE_CHUNK_FC1
+#define LMOE_CHUNK_FC1 4     // fc1 when z is re-rounded: smaller partial sums, a smaller margin
+#endif
+
 // The exact re-rounding list of a relu2 activation problem (see rr_flag).
 void set_act_recheck(const Ctx& c, GemmProblem& pr, int* count) {
     const double tau = c.h->act_tau, c0 = c.h->act_c0, c1 = c.h->act_c1;
@@ -424,8 +440,8 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
                              make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is)};
         pr[0].kdim[0] = H;
         pr[1].kdim[0] = H;
-        // fc1 in chunks of 4 k-blocks when z is re-rounded: half the fp32 error, half the list
-        if (zcheck) pr[0].chunk_kb = 4;
+        // fc1 in short chunks when z is re-rounded: a smaller fp32 error, a shorter list
+        if (zcheck) pr[0].chunk_kb = LMOE_CHUNK_FC1;
         if (act_rr) set_act_recheck(c, pr[1], &c.st->asflagged);
         pr[0].a_ptr[0] = xa;
         pr[0].b_ptr[0] = h->w.fc1_w;
@@ -476,6 +492,7 @@ lmoe_status stage_experts(Ctx& c, const void* rows, long long n, const float* ro
         pr.kdim[0] = L;
         pr.b_rows_per_expert = I;
         pr.expert_mod = expert_mod;
+        pr.chunk_kb = LMOE_CHUNK_UP;
         if (act_rr) set_act_recheck(c, pr, &c.st->aeflagged);
         pr.a_ptr[0] = rows;
         pr.b_ptr[0] = h->w.up_w;
@@ -501,6 +518,7 @@ lmoe_status stage_experts(Ctx& c, const void* rows, long long n, const float* ro
         pr.kdim[0] = I;
         pr.b_rows_per_expert = L;
         pr.expert_mod = expert_mod;
+        pr.chunk_kb = LMOE_CHUNK_DOWN;
         pr.row_scale = row_w;
         pr.a_ptr[0] = a_buf;
         pr.b_ptr[0] = h->w.down_w;
@@ -534,6 +552,7 @@ lmoe_status stage_back(Ctx& c, const float* o, float* y, const uint16_t* resid) 
     mark(c, 6);
     {
         GemmProblem pr = make_problem(0, p.T, H, EPI_F32, y, H);
+        pr.chunk_kb = LMOE_CHUNK_OUT;
         pr.nseg = 2;
         pr.kdim[0] = L;
         pr.kdim[1] = Is;

@@ -69,6 +69,53 @@ __device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
     e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
 }
 
+// Error-free dot product of one lane's share of two bf16 rows (uint4 = 8 values,
+// vectors k = lane, lane + 32, ... < K8): the exact products are summed into
+// four independent hi + lo chains (one per bf16 pair of the vector, so the
+// TwoSum dependency chains interleave), then merged without error. Returns the
+// lane's pair; the caller reduces the warp.
+template <typename LoadA>
+__device__ __forceinline__ void dot_pairs(LoadA load_a, const uint4* __restrict__ wr, int K8, int lane, float& hi,
+                                          float& lo) {
+    float h[4] = {0.f, 0.f, 0.f, 0.f}, l[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = lane; k < K8; k += 32) {
+        const uint4 a = load_a(k), b = __ldg(wr + k);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float e;
+            two_sum(h[j], __fmul_rn(__uint_as_float(av[j] << 16), __uint_as_float(bv[j] << 16)), h[j], e);
+            l[j] = __fadd_rn(l[j], e);
+            two_sum(h[j], __fmul_rn(__uint_as_float(av[j] & 0xFFFF0000u), __uint_as_float(bv[j] & 0xFFFF0000u)), h[j],
+                    e);
+            l[j] = __fadd_rn(l[j], e);
+        }
+    }
+    hi = h[0];
+    lo = l[0];
+#pragma unroll
+    for (int j = 1; j < 4; ++j) {
+        float e;
+        two_sum(hi, h[j], hi, e);
+        lo = __fadd_rn(__fadd_rn(lo, l[j]), e);
+    }
+}
+
+// Warp reduction of the lanes' pairs (error-free merges), then the
+// renormalised pair: hi = fl(hi + lo), lo the exact remainder.
+__device__ __forceinline__ void warp_reduce_pair(float& hi, float& lo) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float oh = __shfl_xor_sync(0xffffffffu, hi, o), ol = __shfl_xor_sync(0xffffffffu, lo, o);
+        float e;
+        two_sum(hi, oh, hi, e);
+        lo = __fadd_rn(__fadd_rn(lo, ol), e);
+    }
+    float rest;
+    two_sum(hi, lo, hi, rest);
+    lo = rest;
+}
+
 // Nearest-even bf16 of hi + lo, where hi = fl32(hi + lo) and |lo| <= ulp(hi)/2.
 // Every bf16 rounding midpoint is an fp32 number, so hi + lo lies on the same
 // side of each midpoint as hi unless hi is a midpoint itself; then the sign of
@@ -164,30 +211,10 @@ __global__ void __launch_bounds__(256) k_recheck_rows(const uint16_t* __restrict
             const int2 ent = list[e];
             if (!lmoe_check((unsigned)ent.y < (unsigned)w_rows, err)) continue;
             const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)ent.y * K);
-            float hi = 0.f, lo = 0.f;
-            for (int k = lane; k < K8; k += 32) {
-                const uint4 a = xs[k], b = __ldg(wr + k);
-                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float err2;
-                    two_sum(hi, __fmul_rn(__uint_as_float(av[j] << 16), __uint_as_float(bv[j] << 16)), hi, err2);
-                    lo = __fadd_rn(lo, err2);
-                    two_sum(hi, __fmul_rn(__uint_as_float(av[j] & 0xFFFF0000u), __uint_as_float(bv[j] & 0xFFFF0000u)),
-                            hi, err2);
-                    lo = __fadd_rn(lo, err2);
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float oh = __shfl_xor_sync(0xffffffffu, hi, o), ol = __shfl_xor_sync(0xffffffffu, lo, o);
-                float err2;
-                two_sum(hi, oh, hi, err2);
-                lo = __fadd_rn(__fadd_rn(lo, ol), err2);
-            }
-            float rest;
-            two_sum(hi, lo, hi, rest);
-            if (lane == 0) out[(size_t)rt.x * ldo + ent.y] = bf16_rn_of_pair(hi, rest);
+            float hi, lo;
+            dot_pairs([&](int k) { return xs[k]; }, wr, K8, lane, hi, lo);
+            warp_reduce_pair(hi, lo);
+            if (lane == 0) out[(size_t)rt.x * ldo + ent.y] = bf16_rn_of_pair(hi, lo);
         }
     }
 }
@@ -215,36 +242,16 @@ __global__ void __launch_bounds__(256) k_recheck(const uint16_t* __restrict__ A,
         if (!lmoe_check((unsigned)e.x < (unsigned)a_rows && (unsigned)e.y < (unsigned)w_rows, err)) continue;
         const uint4* xr = reinterpret_cast<const uint4*>(A + (size_t)e.x * K);
         const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)e.y * K);
-        float hi = 0.f, lo = 0.f;
-        for (int k = lane; k < K8; k += 32) {
-            const uint4 a = __ldg(xr + k), b = __ldg(wr + k);
-            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float err2;
-                two_sum(hi, __fmul_rn(__uint_as_float(av[j] << 16), __uint_as_float(bv[j] << 16)), hi, err2);
-                lo = __fadd_rn(lo, err2);
-                two_sum(hi, __fmul_rn(__uint_as_float(av[j] & 0xFFFF0000u), __uint_as_float(bv[j] & 0xFFFF0000u)),
-                        hi, err2);
-                lo = __fadd_rn(lo, err2);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float oh = __shfl_xor_sync(0xffffffffu, hi, o), ol = __shfl_xor_sync(0xffffffffu, lo, o);
-            float err2;
-            two_sum(hi, oh, hi, err2);
-            lo = __fadd_rn(__fadd_rn(lo, ol), err2);
-        }
-        float rest;
-        two_sum(hi, lo, hi, rest);  // renormalise: hi = fl(hi + lo), rest the exact remainder
+        float hi, lo;
+        dot_pairs([&](int k) { return __ldg(xr + k); }, wr, K8, lane, hi, lo);
+        warp_reduce_pair(hi, lo);
         if (lane == 0) {
             uint16_t r;
             if (kRelu2) {
-                const double h = (double)hi + (double)rest;  // exact: 48 significant bits at most
+                const double h = (double)hi + (double)lo;  // exact: 48 significant bits at most
                 r = h > 0.0 ? bf16_rn_from_double(h * h) : (uint16_t)0;
             } else {
-                r = bf16_rn_of_pair(hi, rest);
+                r = bf16_rn_of_pair(hi, lo);
             }
             out[(size_t)e.x * ldo + (e.y % ldo)] = r;
         }
