@@ -293,9 +293,12 @@ lmoe_status latentmoe_read_stats(const lmoe_handle* h, const void* ws, lmoe_stat
  * re-rounding; flag_list: int32 ids of the tokens re-decided in fp64
  * (lmoe_stats.flagged_tokens of them); perm [T*k] int32: token of each row in
  * expert order; slot [T, k] int32: row in expert order of each (token, j);
- * total = latentmoe_workspace_size(T). */
+ * total = latentmoe_workspace_size(T); offsets [E + 1] int32: first row of
+ * each expert in expert order; act_e [T*k, I] bf16 expert activations
+ * relu2(z W_up^T) in expert order and act_s [T, Is] bf16 shared-expert
+ * activations (bf16 mode, after latentmoe_forward). */
 typedef struct {
-    size_t logits_f32, z_f32, z, flag_list, perm, slot, total;
+    size_t logits_f32, z_f32, z, flag_list, perm, slot, total, offsets, act_e, act_s;
 } lmoe_ws_layout;
 lmoe_status latentmoe_workspace_layout(const lmoe_handle* h, int T, lmoe_ws_layout* out);
 

@@ -58,7 +58,8 @@ class lmoe_stats(ctypes.Structure):
 
 
 class lmoe_ws_layout(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_size_t) for n in ("logits_f32", "z_f32", "z", "flag_list", "perm", "slot", "total")]
+    _fields_ = [(n, ctypes.c_size_t) for n in ("logits_f32", "z_f32", "z", "flag_list", "perm", "slot", "total",
+                                              "offsets", "act_e", "act_s")]
 
 
 class LmoeError(RuntimeError):

@@ -785,6 +785,9 @@ lmoe_status latentmoe_workspace_layout(const lmoe_handle* h, int T, lmoe_ws_layo
     out->perm = p.perm;
     out->slot = p.slot;
     out->total = p.total;
+    out->offsets = p.offsets;
+    out->act_e = p.aperm;
+    out->act_s = p.as;
     return LMOE_OK;
 }
 

@@ -58,6 +58,51 @@ __device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
     return h | (h << 16);
 }
 
+// The same conversion with the block scale folded into the byte tables: t
+// holds, for one E4M3 scale s, the high bytes (t.x: magnitudes 0..3, t.y:
+// 4..7) and low bytes (t.z, t.w) of the bf16 values of s * {0, 0.5, 1, 1.5,
+// 2, 3, 4, 6}. Those products are exact in bf16 (at most 6 significant bits),
+// so the result equals e2m1x8_to_bf16(c, s) bit for bit, signs and zeros
+// included, without the four multiplies.
+__device__ __forceinline__ uint4 e2m1x8_to_bf16_scaled(uint32_t c, const uint4& t) {
+    const uint32_t mag = c & 0x77777777u;
+    const uint32_t d = c << 4;
+    const uint32_t mhi = mag >> 16;
+    const uint32_t h0 = prmt(t.x, t.y, mag) ^ (prmt(d, c, 0x5140u) & 0x80808080u);
+    const uint32_t l0 = prmt(t.z, t.w, mag);
+    const uint32_t h1 = prmt(t.x, t.y, mhi) ^ (prmt(d, c, 0x7362u) & 0x80808080u);
+    const uint32_t l1 = prmt(t.z, t.w, mhi);
+    uint4 o;
+    o.x = prmt(l0, h0, 0x5140u);
+    o.y = prmt(l0, h0, 0x7362u);
+    o.z = prmt(l1, h1, 0x5140u);
+    o.w = prmt(l1, h1, 0x7362u);
+    return o;
+}
+
+// Byte tables of e2m1x8_to_bf16_scaled for the E4M3 scale byte b: the bf16
+// products s * m of the eight magnitudes m, signs included (0 * s is -0 for a
+// negative s). A code's sign bit flips its product's sign (xor), which is
+// what the multiply by s gives for every code, -0 and negative scales
+// included.
+__device__ __forceinline__ uint4 e4m3_scaled_table(uint32_t b) {
+    const uint32_t s2 = e4m3_to_bf16x2(b);
+    uint32_t hi[8], lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        constexpr uint32_t kMag[8] = {0x0000u, 0x3F00u, 0x3F80u, 0x3FC0u, 0x4000u, 0x4040u, 0x4080u, 0x40C0u};
+        const uint32_t v = mul_bf16x2(kMag[j] | (kMag[j] << 16), s2) & 0xFFFFu;
+        hi[j] = v >> 8;
+        lo[j] = v & 0xFFu;
+    }
+    uint4 t;
+    t.x = hi[0] | (hi[1] << 8) | (hi[2] << 16) | (hi[3] << 24);
+    t.y = hi[4] | (hi[5] << 8) | (hi[6] << 16) | (hi[7] << 24);
+    t.z = lo[0] | (lo[1] << 8) | (lo[2] << 16) | (lo[3] << 24);
+    t.w = lo[4] | (lo[5] << 8) | (lo[6] << 16) | (lo[7] << 24);
+    return t;
+}
+
 // ------------------------------------------------------------------------------
 // The dequantised weights live in TMEM: the tensor core takes its A operand
 // (128 weight rows x K) from TMEM, so the bf16 weight tile never passes through
@@ -71,13 +116,23 @@ __device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
 // works on every stage, group g converting the stage's k-blocks j with
 // j % G == g, so a stage's conversion is spread over all G x 4 warps (one
 // group per stage made each stage a long serial chain per thread).
-// TMEM columns: [0, 256) accumulator chunk buffers, [256, 512)
-// AS slots of KB bf16 weight tiles. The shared-memory ring (codes, scales,
-// token tiles) is deeper than the slot ring, so copies run far ahead of the
-// conversions: before it overwrites slot c % AS, the conversion of stage c
-// waits for the MMA of stage c - AS, the slot's last reader, on that stage's
-// `empty` barrier (no barrier is added to the MMA's path).
-template <int BN, int STAGES, int KB, int G, int AS>
+// TMEM columns: [0, NB * NI * BN) accumulator chunk buffers (one accumulator
+// per MMA issuer), then AS slots of KB bf16 weight tiles (32 columns each).
+// The shared-memory ring (codes, scales, token tiles) is deeper than the slot
+// ring, so copies run far ahead of the conversions: before it overwrites slot
+// c % AS, the conversion of stage c waits for the MMA of stage c - AS, the
+// slot's last reader, on that stage's `empty` barrier (no barrier is added to
+// the MMA's path).
+// Template parameters: BN tokens per tile, STAGES shared-memory stages of KB
+// k-blocks, G dequantisation warp groups, AS TMEM weight slots, NB accumulator
+// chunk buffers, NI MMA-issuing warps (issuer i takes the k-blocks j % NI == i
+// of a stage), SL conversion through per-scale byte tables.
+// At decode sizes a 128 x 32 x 16 MMA occupies the tensor core ~48 cycles
+// whatever its N (up to 64), so a stage of four k-blocks has ~780 cycles of
+// tensor time; the measured stage takes ~2000, spent on the conversion
+// (~1300 cycles of ALU work per warp), the MMA issuer's barrier round trips
+// and its slower issue next to the converting warps.
+template <int BN, int STAGES, int KB, int G, int AS, int NB, int NI, bool SL>
 struct Fp4TmShape {
     using T = Shape<BN, true>;
     static constexpr int kTokBytes = BN * kBK * 2;
@@ -85,25 +140,26 @@ struct Fp4TmShape {
     static constexpr int kOffSf = kOffCodes + KB * 4096;
     static constexpr int kStageBytes = (kOffSf + KB * 512 + 1023) & ~1023;
     static constexpr int kTxBytes = KB * (kTokBytes + 4096 + 512);
-    static constexpr int kBufs = 256 / BN;           // accumulator chunk buffers in columns [0, 256)
-    static constexpr uint32_t kColA = 256;           // first column of the weight tiles
+    static constexpr int kBufs = NB;                 // accumulator chunk buffers, one accumulator per MMA issuer
+    static constexpr uint32_t kColA = NB * NI * BN;  // first column of the weight tiles
     static constexpr int kDeqWarps = 4 * G;
-    static constexpr int kThreads = 64 + 32 * (T::kEpiWarps + kDeqWarps);
+    static constexpr int kThreads = 32 * (1 + NI + T::kEpiWarps + kDeqWarps);
     static constexpr int kBarBytes = 1024;
     static constexpr int kBars = 3 * STAGES + 2 * kBufs + 1;
-    static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStageBytes + kBarBytes + 1024;
-    static_assert(AS * KB * 32 <= 256 && AS <= STAGES, "weight tiles fit TMEM columns [256, 512)");
+    static constexpr int kLutBytes = SL ? 256 * 16 : 256 * 4;  // per-scale byte tables, or bf16 scales
+    static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStageBytes + kBarBytes + kLutBytes;
+    static_assert(kColA + AS * KB * 32 <= 512 && AS <= STAGES, "accumulators and weight tiles fit TMEM");
     static_assert(kBars * 8 + 4 <= kBarBytes, "barrier area");
-    static_assert(KB % G == 0 && T::kChunkKB % KB == 0, "groups / chunks");
+    static_assert(KB % G == 0 && KB % NI == 0 && T::kChunkKB % KB == 0 && (NI == 1 || NI == 2), "groups / chunks");
     static_assert(kSmem <= 232448 && STAGES <= 32, "shared memory");
 };
 
-template <int BN, int STAGES, int KB, int G, int AS>
-__global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1)
+template <int BN, int STAGES, int KB, int G, int AS, int NB, int NI, bool SL>
+__global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS, NB, NI, SL>::kThreads, 1)
     k_gemm_nvfp4_tm(const __grid_constant__ TcParams P) {
-    using F = Fp4TmShape<BN, STAGES, KB, G, AS>;
+    using F = Fp4TmShape<BN, STAGES, KB, G, AS, NB, NI, SL>;
     using S = typename F::T;
-    constexpr int NB = F::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
+    constexpr int CK = S::kChunkKB, CW = S::kColsPerThread;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
@@ -121,18 +177,23 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&deq[s], 4 * G);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], NI);
         }
         for (int b = 0; b < NB; ++b) {
-            mbar_init(&cfull[b], 1);
+            mbar_init(&cfull[b], NI);
             mbar_init(&cempty[b], S::kEpiWarps);
         }
-        mbar_init(done, 1);
+        mbar_init(done, NI);
         fence_mbar_init();
     }
-    const int dq0 = 2 + S::kEpiWarps;  // first dequantisation warp
+    const int dq0 = 1 + NI + S::kEpiWarps;  // first dequantisation warp
     if (warp >= dq0)
-        for (int b = threadIdx.x - 32 * dq0; b < 256; b += 32 * F::kDeqWarps) scale_lut[b] = e4m3_to_bf16x2((uint32_t)b);
+        for (int b = threadIdx.x - 32 * dq0; b < 256; b += 32 * F::kDeqWarps) {
+            if constexpr (SL)
+                reinterpret_cast<uint4*>(scale_lut)[b] = e4m3_scaled_table((uint32_t)b);
+            else
+                scale_lut[b] = e4m3_to_bf16x2((uint32_t)b);
+        }
     if (warp == 0 && lane == 0)
         for (int i = 0; i < P.nmaps; ++i) prefetch_tmap(&P.maps[i]);
     if (warp == 1) {
@@ -177,9 +238,11 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
         }
         for (int s = 0; s < STAGES; ++s)
             if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp >= 1 && warp <= NI && lane == 0) {
+        // ------------------------------------------------ MMA issuers: issuer i takes the k-blocks
+        // j % NI == i of every stage into its own accumulator of the chunk buffer
         constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+        const int iss = warp - 1;
         uint32_t c = 0, bphase = 0;
         int buf = 0;
         bool ok = true;
@@ -190,7 +253,7 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+                const uint32_t d = tmem_base + (uint32_t)((buf * NI + iss) * BN);
                 const int kb1 = min(kb_n, kb0 + CK);
                 for (int kb = kb0; kb < kb1; kb += KB, ++c) {
                     const int s = (int)(c % STAGES);
@@ -202,13 +265,14 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
                     tc_fence_after();
                     const uint8_t* st = smem + s * F::kStageBytes;
 #pragma unroll
-                    for (int j = 0; j < KB; ++j) {
+                    for (int jj = 0; jj < KB / NI; ++jj) {
+                        const int j = jj * NI + iss;
                         const uint32_t a = tmem_base + F::kColA + (uint32_t)(((c % AS) * KB + j) * 32);
                         const uint64_t bdesc = sdesc_sw128(smem_u32(st + j * F::kTokBytes));
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk)
                             umma_bf16_tmem_a(d, a + (uint32_t)(kk * 8), bdesc + (uint64_t)(kk * 2), idesc,
-                                             (kb + j > kb0 || kk > 0) ? 1u : 0u);
+                                             (kb + j - iss > kb0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -251,16 +315,26 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
                     const uint8_t* codes = st + F::kOffCodes + j * 4096 + row * 32;
                     const uint4 c0 = ld_shared_v4(codes), c1 = ld_shared_v4(codes + 16);
                     const uint32_t sb = ld_shared_u32(st + F::kOffSf + j * 512 + row * 4);
-                    const uint32_t s0 = ld_shared_u32(scale_lut + (sb & 0xFFu));
-                    const uint32_t s1 = ld_shared_u32(scale_lut + ((sb >> 8) & 0xFFu));
-                    const uint32_t s2 = ld_shared_u32(scale_lut + ((sb >> 16) & 0xFFu));
-                    const uint32_t s3 = ld_shared_u32(scale_lut + (sb >> 24));
+                    uint4 os[8];
+                    if constexpr (SL) {
+                        const uint4* tl = reinterpret_cast<const uint4*>(scale_lut);
+                        const uint4 t0 = ld_shared_v4(tl + (sb & 0xFFu)), t1 = ld_shared_v4(tl + ((sb >> 8) & 0xFFu));
+                        const uint4 t2 = ld_shared_v4(tl + ((sb >> 16) & 0xFFu)), t3 = ld_shared_v4(tl + (sb >> 24));
+                        os[0] = e2m1x8_to_bf16_scaled(c0.x, t0), os[1] = e2m1x8_to_bf16_scaled(c0.y, t0);
+                        os[2] = e2m1x8_to_bf16_scaled(c0.z, t1), os[3] = e2m1x8_to_bf16_scaled(c0.w, t1);
+                        os[4] = e2m1x8_to_bf16_scaled(c1.x, t2), os[5] = e2m1x8_to_bf16_scaled(c1.y, t2);
+                        os[6] = e2m1x8_to_bf16_scaled(c1.z, t3), os[7] = e2m1x8_to_bf16_scaled(c1.w, t3);
+                    } else {
+                        const uint32_t s0 = ld_shared_u32(scale_lut + (sb & 0xFFu));
+                        const uint32_t s1 = ld_shared_u32(scale_lut + ((sb >> 8) & 0xFFu));
+                        const uint32_t s2 = ld_shared_u32(scale_lut + ((sb >> 16) & 0xFFu));
+                        const uint32_t s3 = ld_shared_u32(scale_lut + (sb >> 24));
+                        os[0] = e2m1x8_to_bf16(c0.x, s0), os[1] = e2m1x8_to_bf16(c0.y, s0);
+                        os[2] = e2m1x8_to_bf16(c0.z, s1), os[3] = e2m1x8_to_bf16(c0.w, s1);
+                        os[4] = e2m1x8_to_bf16(c1.x, s2), os[5] = e2m1x8_to_bf16(c1.y, s2);
+                        os[6] = e2m1x8_to_bf16(c1.z, s3), os[7] = e2m1x8_to_bf16(c1.w, s3);
+                    }
                     uint32_t w[32];
-                    const uint4 o0 = e2m1x8_to_bf16(c0.x, s0), o1 = e2m1x8_to_bf16(c0.y, s0);
-                    const uint4 o2 = e2m1x8_to_bf16(c0.z, s1), o3 = e2m1x8_to_bf16(c0.w, s1);
-                    const uint4 o4 = e2m1x8_to_bf16(c1.x, s2), o5 = e2m1x8_to_bf16(c1.y, s2);
-                    const uint4 o6 = e2m1x8_to_bf16(c1.z, s3), o7 = e2m1x8_to_bf16(c1.w, s3);
-                    const uint4 os[8] = {o0, o1, o2, o3, o4, o5, o6, o7};
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         w[4 * i] = os[i].x;
@@ -276,10 +350,10 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
                 if (lane == 0) mbar_arrive(&deq[s]);
             }
         }
-    } else if (warp >= 2) {
+    } else if (warp > NI) {
         // ------------------------------------------------ epilogue (as the bf16 swap tiles)
         const GemmProblem& pr = P.prob[0];
-        const int ew = warp - 2;
+        const int ew = warp - 1 - NI;
         const int q = warp & 3;
         const int c0 = (ew >> 2) * CW;
         const int lane_row = q * 32 + lane;
@@ -297,18 +371,21 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
                     break;
                 }
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0);
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NI * BN + c0);
 #pragma unroll
-                for (int cc = 0; cc < CW; cc += 32) {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld16(taddr + (uint32_t)cc, r0);
-                    if (cc + 16 < CW) tmem_ld16(taddr + (uint32_t)(cc + 16), r1);
-                    tmem_ld_wait();
+                for (int na = 0; na < NI; ++na) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[cc + i] += __uint_as_float(r0[i]);
-                    if (cc + 16 < CW) {
+                    for (int cc = 0; cc < CW; cc += 32) {
+                        uint32_t r0[16], r1[16];
+                        tmem_ld16(taddr + (uint32_t)(na * BN + cc), r0);
+                        if (cc + 16 < CW) tmem_ld16(taddr + (uint32_t)(na * BN + cc + 16), r1);
+                        tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[cc + 16 + i] += __uint_as_float(r1[i]);
+                        for (int i = 0; i < 16; ++i) acc[cc + i] += __uint_as_float(r0[i]);
+                        if (cc + 16 < CW) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) acc[cc + 16 + i] += __uint_as_float(r1[i]);
+                        }
                     }
                 }
                 tc_fence_before();
@@ -330,13 +407,13 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS>::kThreads, 1
     }
 }
 
-template <int BN, int STAGES, int KB, int G, int AS>
+template <int BN, int STAGES, int KB, int G, int AS, int NB, int NI, bool SL>
 cudaError_t launch_nvfp4_tm(const TcParams& P, int grid, cudaStream_t s) {
-    using F = Fp4TmShape<BN, STAGES, KB, G, AS>;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS>,
+    using F = Fp4TmShape<BN, STAGES, KB, G, AS, NB, NI, SL>;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS, NB, NI, SL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F::kSmem);
     if (e != cudaSuccess) return e;
-    k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS><<<grid, F::kThreads, F::kSmem, s>>>(P);
+    k_gemm_nvfp4_tm<BN, STAGES, KB, G, AS, NB, NI, SL><<<grid, F::kThreads, F::kSmem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -352,10 +429,11 @@ cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmP
     const int grid = tc_num_sms();
     switch (bn) {
         case kDecodeTN:
-            // four k-blocks per stage where K allows (a multiple of 256), else two
-            if ((probs[0].kdim[0] / kBK) % 4 == 0) return launch_nvfp4_tm<kDecodeTN, 5, 4, 2, 2>(P, grid, s);
-            return launch_nvfp4_tm<kDecodeTN, 8, 2, 2, 4>(P, grid, s);
-        case 128: return launch_nvfp4_tm<128, 5, 2, 1, 4>(P, grid, s);
+            // four k-blocks per stage where K allows (a multiple of 256), else two; the decode
+            // tiles read the conversion's per-scale byte tables
+            if ((probs[0].kdim[0] / kBK) % 4 == 0) return launch_nvfp4_tm<kDecodeTN, 5, 4, 2, 2, 8, 1, true>(P, grid, s);
+            return launch_nvfp4_tm<kDecodeTN, 8, 2, 2, 4, 8, 1, true>(P, grid, s);
+        case 128: return launch_nvfp4_tm<128, 5, 2, 1, 4, 2, 1, false>(P, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -4,6 +4,10 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#ifndef LMOE_WAIT_TEST
+#define LMOE_WAIT_TEST 1
+#endif
+
 namespace lmoe {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -36,10 +40,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the same phase (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: polls at most `limit` times; every 4096 polls it also looks at
 // the kernel-wide abort word so that one role's timeout releases the others.
-// On running out it records LMOE_ERR_TIMEOUT (5) and returns false.
+// On running out it records LMOE_ERR_TIMEOUT (5) and returns false. A phase
+// that has already completed is taken by one non-blocking test.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned limit, int* err) {
+#if LMOE_WAIT_TEST
+    if (mbar_test_wait(bar, parity)) return true;
+#endif
     for (unsigned i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 4095u) == 4095u && *(volatile int*)err != 0) return false;

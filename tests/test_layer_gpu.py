@@ -336,6 +336,66 @@ def test_z_fp32_error_is_far_inside_the_rerounding_margin():
     assert flips == 0
 
 
+DEFAULT_ACT_TAU = 2.0       # LMOE_OPT_ACT_RECHECK_TAU default (2000, in units of 1e-3)
+
+
+def _exact_relu2(shape_k_n, rows_bits, w_bits):
+    """Exact h = rows . W^T (the oracle's dot product; rows are bf16, so its rounding of the
+    input row is the identity) and the exact rounding of relu(h)^2."""
+    K, N = shape_k_n
+    cfg = oracle.make_cfg(replace(TINY, H=K, L=N, x_f32=False))
+    h = oracle.latent(cfg, rows_bits, w_bits)
+    a = np.vectorize(oracle.round_bf16)(np.maximum(h, 0.0) ** 2)
+    return h, (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_activations_above_tau_are_exact_roundings():
+    """The expert and shared-expert activations a = bf16(relu(h)^2) with h above tau (2.0) are
+    re-rounded exactly when their fp32 value lies near a rounding midpoint, so on the
+    16384-token Ultra batch every such element must equal the exact rounding bit for bit:
+    48 rows of a_e (4 rows of each of 12 experts hit) and 8 rows of a_s. Elements below tau
+    keep the fp32-decided rounding; their share of flips is printed."""
+    import torch
+    shape = ULTRA_PREFILL
+    layer, dev = H.device_layer(shape)
+    T, L, I, Is, A = shape.T, shape.L, shape.I, shape.Is, shape.T * shape.k
+    y = torch.empty((T, shape.H), dtype=torch.float32, device="cuda")
+    layer.forward(dev["x"], y)
+    torch.cuda.synchronize()
+    st = layer.stats()
+    lay = layer.layout(T)
+    offs = layer.ws_view(lay.offsets, (shape.E + 1,), torch.int32).cpu().numpy()
+    perm = layer.ws_view(lay.perm, (A,), torch.int32)
+    zb = layer.ws_view(lay.z, (T, L), torch.bfloat16)
+    ae = layer.ws_view(lay.act_e, (A, I), torch.bfloat16)
+    asb = layer.ws_view(lay.act_s, (T, Is), torch.bfloat16)
+    rng = np.random.default_rng(23)
+    hit = np.nonzero(np.diff(offs) >= 4)[0]
+    experts = rng.choice(hit, 12, replace=False)
+    above = below = flips_below = 0
+    for e in experts:
+        rows = offs[e] + rng.choice(offs[e + 1] - offs[e], 4, replace=False)
+        rt = torch.from_numpy(rows.astype(np.int64)).cuda()
+        tok = perm[rt].long()
+        h, ref = _exact_relu2((L, I), H.bf16_to_bits(zb[tok]), H.bf16_to_bits(dev["up_w"][int(e)]))
+        got = H.bf16_to_bits(ae[rt])
+        big = h > DEFAULT_ACT_TAU
+        above += int(big.sum())
+        assert np.array_equal(got[big], ref[big]), "expert %d: a_e above tau differs from the exact rounding" % e
+        below += int((~big).sum())
+        flips_below += int((got[~big] != ref[~big]).sum())
+    toks = np.sort(rng.choice(T, 8, replace=False))
+    hs, ref_s = _exact_relu2((shape.H, Is), H.host_x(shape, dev, toks), H.bf16_to_bits(dev["shared_up_w"]))
+    got_s = H.bf16_to_bits(asb[torch.from_numpy(toks).cuda()])
+    big_s = hs > DEFAULT_ACT_TAU
+    assert np.array_equal(got_s[big_s], ref_s[big_s]), "a_s above tau differs from the exact rounding"
+    print("activations: a_e %d elements above tau exact, %d of %d below tau flipped; a_s %d above tau exact, "
+          "%d of %d below flipped; listed for re-rounding: a_e %d, a_s %d" %
+          (above, flips_below, below, int(big_s.sum()), int((got_s[~big_s] != ref_s[~big_s]).sum()),
+           int((~big_s).sum()), st.ae_rechecked, st.as_rechecked))
+    assert above > 0 and big_s.any() and st.ae_rechecked > 0 and st.as_rechecked > 0
+
+
 # ---------------------------------------------------------------- ties
 TIES = LayerShape("ties", T=257, H=512, L=256, E=64, k=5, G=4, Gk=2, I=384, Is=640)
 
