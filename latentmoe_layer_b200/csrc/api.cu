@@ -266,6 +266,9 @@ cudaError_t run_gemm_nvfp4(Ctx& c, GemmProblem* pr, const Operand& act) {
 #ifndef LMOE_CHUNK_FC1
 #define LMOE_CHUNK_FC1 4     // fc1 when z is re-rounded: smaller partial sums, a smaller margin
 #endif
+#ifndef LMOE_CHUNK_SHARED_UP
+#define LMOE_CHUNK_SHARED_UP 4  // shared up (a_s, K = H) when its activations are re-rounded
+#endif
 
 // The exact re-rounding list of a relu2 activation problem (see rr_flag).
 void set_act_recheck(const Ctx& c, GemmProblem& pr, int* count) {
@@ -442,7 +445,10 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         pr[1].kdim[0] = H;
         // fc1 in short chunks when z is re-rounded: a smaller fp32 error, a shorter list
         if (zcheck) pr[0].chunk_kb = LMOE_CHUNK_FC1;
-        if (act_rr) set_act_recheck(c, pr[1], &c.st->asflagged);
+        if (act_rr) {
+            set_act_recheck(c, pr[1], &c.st->asflagged);
+            pr[1].chunk_kb = LMOE_CHUNK_SHARED_UP;
+        }
         pr[0].a_ptr[0] = xa;
         pr[0].b_ptr[0] = h->w.fc1_w;
         pr[1].a_ptr[0] = xa;

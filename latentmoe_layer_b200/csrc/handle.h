@@ -15,8 +15,10 @@ struct lmoe_handle {
     // (1.16e-6 + 0.45e-6 |z| over 524288 elements; the smallest ratio seen is 4.5)
     float zcheck_delta = 6e-6f;
     // LMOE_OPT_ACT_RECHECK_TAU: relu2 activations with h above this are re-rounded exactly when
-    // within the accumulation-error margin (act_c0 + act_c1 h: the largest fp32 error measured at
-    // K = 8192 in chunks of 8 k-blocks) of a bf16 midpoint
+    // within the accumulation-error margin act_c0 + act_c1 h of a bf16 midpoint. The margin is the
+    // largest fp32 error measured at K = 8192 in TMEM chunks of 8 k-blocks; the shared up GEMM
+    // (K = H = 8192) runs in chunks of 4 (measured on fc1, the same x and K: 1.16e-6 + 0.45e-6 h,
+    // so the margin is 1.4-2x), the expert up GEMM (K = L = 2048) has a quarter of the chunks
     float act_tau = 2.0f;
     float act_c0 = 1.6e-6f, act_c1 = 0.9e-6f;
     unsigned spin_limit = 1u << 24;

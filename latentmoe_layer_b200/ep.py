@@ -18,6 +18,18 @@ Per forward, on every rank:
   4 experts  this rank's experts on the received rows, in arrival order
   5 return   all-to-all of the fp32 results back to the senders
   6 back     combine in ascending expert id and fc2 + shared down -> y
+
+Costs this design accepts:
+  - The return leg carries fp32 rows, 4*L bytes per assignment (8 KB at L = 2048)
+    against 2*L on the bf16 dispatch: the expert outputs o_e are fp32 up to the
+    combine's single rounding, so a bf16 return would add a rounding the layer
+    does not have. The exchange moves 6*L bytes per assignment in all, still
+    under half of what hidden-width rows would (2*H out, 4*H back at H = 4*L).
+  - exchange_plan reads the split sizes on the host (one device-to-host copy of
+    P integers and the wait for it, per forward): all_to_all_single takes host
+    split sizes. An exchange at fixed capacity would need no host read but move
+    up to min(k, E/P) * T rows to every rank, P times the mean at the Ultra
+    shape.
 """
 from __future__ import annotations
 
