@@ -343,17 +343,21 @@ lmoe_status validate_call(lmoe_handle* h, const void* x, int T, void* ws, size_t
     return LMOE_OK;
 }
 
-// Routing stages 1-4. Writes idx/w/counts into the workspace and, if given,
-// the caller's outputs.
-lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
+// Routing, first part: the statistics reset and the fp32 router logits (tensor
+// cores), unless every token is decided in fp64.
+bool route_fp64_all(const Ctx& c) {
+    const lmoe_config& cf = c.h->cfg;
+    return c.h->fp64_all || cf.mode == LMOE_MODE_FP32 || cf.x_dtype == LMOE_FP32 || cf.num_experts % 64 != 0 ||
+           c.simt;
+}
+
+lmoe_status route_head(Ctx& c, const void* x) {
     lmoe_handle* h = c.h;
     const lmoe_config& cf = h->cfg;
     const Plan& p = *c.p;
     char* ws = c.ws;
-    const bool fp64_all = h->fp64_all || cf.mode == LMOE_MODE_FP32 || cf.x_dtype == LMOE_FP32 ||
-                          cf.num_experts % 64 != 0 || c.simt;
     LMOE_TRY(cudaMemsetAsync(ws + p.stats, 0, sizeof(WsStats), c.s));
-    if (!fp64_all) {
+    if (!route_fp64_all(c)) {
         GemmProblem pr = make_problem(0, p.T, cf.num_experts, EPI_F32, ws + p.logits, cf.num_experts);
         pr.kdim[0] = cf.hidden;
         Operand a[1][2] = {{{x, p.T}, {nullptr, 0}}};
@@ -361,6 +365,19 @@ lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int3
         Ctx rc = c;
         rc.decode = c.decode && cf.num_experts % 128 == 0;
         LMOE_LAUNCH(1, run_gemm(rc, &pr, 1, a, b, false));
+    }
+    return LMOE_OK;
+}
+
+// Routing, second part: selection with the near-edge flags, the fp64
+// re-decision of the flagged tokens (or of every token), the counting sort.
+// Writes idx/w/counts into the workspace and, if given, the caller's outputs.
+lmoe_status route_tail(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const Plan& p = *c.p;
+    char* ws = c.ws;
+    if (!route_fp64_all(c)) {
         LMOE_LAUNCH(1, launch_router_select(h, p, ws, false, c.s));
         LMOE_LAUNCH(1, launch_router_logits64(h, x, p, ws, false, c.s));
         LMOE_LAUNCH(1, launch_router_select64(h, p, ws, false, c.s));
@@ -374,6 +391,20 @@ lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int3
                                     idx_out, w_out, (long long)p.T * cf.top_k, h->num_sms, c.s));
     return LMOE_OK;
 }
+
+// Routing stages 1-4 in order on the call's stream.
+lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
+    lmoe_status s = route_head(c, x);
+    if (s != LMOE_OK) return s;
+    return route_tail(c, x, idx_out, w_out, counts_out);
+}
+
+// Where the routing tail of a forward writes the caller's copies of its outputs.
+struct RouteOut {
+    int32_t* idx;
+    float* w;
+    int32_t* counts;
+};
 
 Ctx make_ctx(lmoe_handle* h, const Plan& p, void* ws, void* stream) {
     Ctx c;
@@ -412,9 +443,14 @@ __global__ void k_publish_error(const int* derr, int* herr) {
 // [T, H]) the output GEMM adds it: y = resid + layer(x).
 int experts_held(const lmoe_config& c) { return c.local_experts > 0 ? c.local_experts : c.num_experts; }
 
+lmoe_status rerounding(Ctx& c, const void* xa, bool zcheck, bool act_rr);
+
 // Steps 5-6: z = x W_fc1^T and a_s = relu2(x W_su^T) (one launch), then the
-// rows of z in expert order (the permutation of do_route) into zdst.
-lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
+// rows of z in expert order into zdst. The routing tail (route_tail, after
+// route_head on the call's stream) runs here on the handle's second stream, next
+// to the exact re-roundings of z and a_s, which do not read its outputs; the
+// gather, the first reader of the permutation, waits for it.
+lmoe_status stage_front(Ctx& c, const void* x, void* zdst, const RouteOut& ro) {
     lmoe_handle* h = c.h;
     const lmoe_config& cf = h->cfg;
     const Plan& p = *c.p;
@@ -457,6 +493,37 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
         Operand b[2][2] = {{{h->w.fc1_w, L}, {nullptr, 0}}, {{h->w.shared_up_w, Is}, {nullptr, 0}}};
         LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
     }
+    // fork: the routing tail on the second stream once the input GEMM is done (the GEMM keeps
+    // every SM; the tail's kernels share them with the re-roundings)
+    LMOE_TRY(cudaEventRecord(h->ev_fork, c.s));
+    LMOE_TRY(cudaStreamWaitEvent(h->aux, h->ev_fork, 0));
+    Ctx ca = c;
+    ca.s = h->aux;
+    const lmoe_status rs = route_tail(ca, x, ro.idx, ro.w, ro.counts);
+    cudaError_t je = cudaEventRecord(h->ev_join, h->aux);
+    lmoe_status s = rs != LMOE_OK ? rs : rerounding(c, xa, zcheck, act_rr);
+    // join (also after a failure, so that no work of this call is left on the second stream)
+    if (je == cudaSuccess) je = cudaStreamWaitEvent(c.s, h->ev_join, 0);
+    if (s != LMOE_OK) return s;
+    if (je != cudaSuccess) {
+        h->last_cuda_error = (int)je;
+        return LMOE_ERR_CUDA;
+    }
+    mark(c, 2);
+    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, p.T, c.err, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
+                                      reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, h->num_sms, c.s));
+    mark(c, 3);
+    return LMOE_OK;
+}
+
+// The exact re-roundings of the input stage: z (round, list, re-check by row
+// segments) and the shared-expert activations a_s.
+lmoe_status rerounding(Ctx& c, const void* xa, bool zcheck, bool act_rr) {
+    lmoe_handle* h = c.h;
+    const lmoe_config& cf = h->cfg;
+    const Plan& p = *c.p;
+    char* ws_c = c.ws;
+    const int H = cf.hidden, L = cf.latent, Is = cf.shared_inter;
     if (zcheck) {
         const int cap = (int)std::min<long long>((long long)p.T * L, 0x7FFFFFFF);  // T * L < 2^31 (create)
         int2* list = reinterpret_cast<int2*>(ws_c + p.zlist);
@@ -475,10 +542,6 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst) {
                                       static_cast<const uint16_t*>(h->w.shared_up_w), Is, H, c.err, c.alist,
                                       &c.st->asflagged, c.alist_cap, reinterpret_cast<uint16_t*>(ws_c + p.as), Is,
                                       h->num_sms, c.s));
-    mark(c, 2);
-    LMOE_LAUNCH(1, launch_gather_rows(ws_c + p.z, p.T, c.err, zdst, reinterpret_cast<const int*>(ws_c + p.perm), p.A,
-                                      reinterpret_cast<const int*>(ws_c + p.offsets) + E, L * act, h->num_sms, c.s));
-    mark(c, 3);
     return LMOE_OK;
 }
 
@@ -586,10 +649,10 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
     mark(c, 0);
     if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
                                                 reinterpret_cast<uint16_t*>(const_cast<void*>(x)), h->num_sms, c.s));
-    s = do_route(c, x, topk_idx, topk_w, expert_counts);
+    s = route_head(c, x);
     if (s != LMOE_OK) return s;
     mark(c, 1);
-    s = stage_front(c, x, ws_c + p.zperm);
+    s = stage_front(c, x, ws_c + p.zperm, RouteOut{topk_idx, topk_w, expert_counts});
     if (s != LMOE_OK) return s;
     s = stage_experts(c, ws_c + p.zperm, p.A, reinterpret_cast<const float*>(ws_c + p.wperm), ws_c + p.aperm,
                       reinterpret_cast<float*>(ws_c + p.o), 0);
@@ -699,6 +762,14 @@ lmoe_status latentmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe
         return LMOE_ERR_CUDA;
     }
     h->num_sms = tc_num_sms();
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&h->aux, cudaStreamNonBlocking, hi) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+        latentmoe_destroy(h);
+        return LMOE_ERR_CUDA;
+    }
     *out = h;
     return LMOE_OK;
 }
@@ -732,6 +803,9 @@ lmoe_status latentmoe_route(lmoe_handle* h, const void* x, int T, int32_t* topk_
 
 void latentmoe_destroy(lmoe_handle* h) {
     if (!h) return;
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->aux) cudaStreamDestroy(h->aux);
     if (h->herr) cudaFreeHost(h->herr);
     delete h;
 }
@@ -835,10 +909,10 @@ lmoe_status latentmoe_ep_front(lmoe_handle* h, const void* x, int T, void* send_
     Ctx c = make_ctx(h, p, ws, stream);
     h->launches = 0;
     mark(c, 0);
-    s = do_route(c, x, nullptr, nullptr, expert_counts);
+    s = route_head(c, x);
     if (s != LMOE_OK) return s;
     mark(c, 1);
-    s = stage_front(c, x, send_rows);
+    s = stage_front(c, x, send_rows, RouteOut{nullptr, nullptr, expert_counts});
     if (s != LMOE_OK) return s;
     LMOE_TRY(cudaMemcpyAsync(send_w, c.ws + p.wperm, (size_t)p.A * 4, cudaMemcpyDeviceToDevice, c.s));
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);

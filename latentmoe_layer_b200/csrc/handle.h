@@ -27,4 +27,8 @@ struct lmoe_handle {
     int last_cuda_error = 0;           // cudaError_t of the last runtime call that failed (0: none yet)
     void* const* prof_events = nullptr;  // latentmoe_set_profile_events
     int prof_n = 0;
+    // second stream of a forward: the routing tail runs on it next to the exact re-roundings,
+    // forked from and joined back into the caller's stream by the two events
+    cudaStream_t aux = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
