@@ -34,9 +34,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of bf16 tensor peak / HBM BW"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Stages between the library's profile events: "routing" is the router GEMM (the selection, the fp64
-# re-decision and the counting sort run on a second stream inside "input_gemm", next to the exact
-# re-roundings of z and a_s that follow the fc1 + shared up GEMM).
+# Stages between the library's profile events: "routing" is the statistics reset (plus the router GEMM
+# where it cannot join the input GEMM launch); the router logits are the first problem of the fc1 +
+# shared up launch, and the selection, the fp64 re-decision and the counting sort run on a second
+# stream inside "input_gemm", next to the exact re-roundings of z and a_s.
 STAGES = ["routing", "input_gemm", "gather", "expert_up_gemm", "expert_down_gemm", "combine", "output_gemm"]
 
 

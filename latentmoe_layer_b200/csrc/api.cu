@@ -205,22 +205,37 @@ struct Operand {
 cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2], const Operand (*b)[2],
                      bool a_f32_simt) {
     if (c.simt) return launch_gemm_simt(probs, nprob, a_f32_simt, c.r, c.p->A, c.s);
-    int ns[2] = {probs[0].n, nprob > 1 ? probs[1].n : probs[0].n};
+    if (nprob < 1 || nprob > kMaxProblems) return cudaErrorInvalidValue;
+    int ns[kMaxProblems];
     bool swap = c.decode;
-    for (int i = 0; i < nprob; ++i) swap = swap && probs[i].n % 128 == 0;
+    for (int i = 0; i < nprob; ++i) {
+        ns[i] = probs[i].n;
+        swap = swap && probs[i].n % 128 == 0;
+    }
     const int bn = swap ? kDecodeTN : pick_bn(ns, nprob);
     if (bn == 0) return cudaErrorInvalidValue;
     // 256 x 256 tiles on 2-SM pairs (option 4): each CTA of the pair loads 128 rows of B
     const bool pair = !swap && bn == 256 && c.h->gemm_path == 4;
-    CUtensorMap maps[8];
+    CUtensorMap maps[kMaxTensorMaps];
     int nm = 0;
     for (int i = 0; i < nprob; ++i)
         for (int sg = 0; sg < probs[i].nseg; ++sg) {
             const int K = probs[i].kdim[sg];
-            if (!encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? kDecodeTN : kBM))
-                return cudaErrorInvalidValue;
-            probs[i].a_map[sg] = nm++;
-            if (!encode_bf16(&maps[nm], b[i][sg].ptr, b[i][sg].rows, K, swap ? kBM : pair ? 128 : bn))
+            // problems that read the same activation matrix share its map
+            int am = -1;
+            for (int j = 0; j < i && am < 0; ++j)
+                if (probs[j].nseg == 1 && a[j][0].ptr == a[i][sg].ptr && a[j][0].rows == a[i][sg].rows &&
+                    probs[j].kdim[0] == K)
+                    am = probs[j].a_map[0];
+            if (am < 0) {
+                if (nm >= kMaxTensorMaps ||
+                    !encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? kDecodeTN : kBM))
+                    return cudaErrorInvalidValue;
+                am = nm++;
+            }
+            probs[i].a_map[sg] = am;
+            if (nm >= kMaxTensorMaps ||
+                !encode_bf16(&maps[nm], b[i][sg].ptr, b[i][sg].rows, K, swap ? kBM : pair ? 128 : bn))
                 return cudaErrorInvalidValue;
             probs[i].b_map[sg] = nm++;
         }
@@ -228,7 +243,8 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
     for (int i = 0; i < nprob && !swap; ++i) {
         const bool f32_out = probs[i].epi == EPI_F32 || probs[i].epi == EPI_SCALE_F32 || probs[i].epi == EPI_RELU2_F32;
         const long long rows = probs[i].grouped ? (long long)c.p->A : probs[i].m_rows;
-        if (probs[i].ldo != probs[i].n || !encode_2d(&maps[nm], probs[i].out, rows, probs[i].n, 32, f32_out)) {
+        if (nm >= kMaxTensorMaps || probs[i].ldo != probs[i].n ||
+            !encode_2d(&maps[nm], probs[i].out, rows, probs[i].n, 32, f32_out)) {
             probs[i].out_map = -1;
             continue;
         }
@@ -343,21 +359,35 @@ lmoe_status validate_call(lmoe_handle* h, const void* x, int T, void* ws, size_t
     return LMOE_OK;
 }
 
-// Routing, first part: the statistics reset and the fp32 router logits (tensor
-// cores), unless every token is decided in fp64.
+// Routing, first part: the statistics reset and, with router_gemm, the fp32
+// router logits (tensor cores), unless every token is decided in fp64.
 bool route_fp64_all(const Ctx& c) {
     const lmoe_config& cf = c.h->cfg;
     return c.h->fp64_all || cf.mode == LMOE_MODE_FP32 || cf.x_dtype == LMOE_FP32 || cf.num_experts % 64 != 0 ||
            c.simt;
 }
 
-lmoe_status route_head(Ctx& c, const void* x) {
+// Whether a forward computes the router logits as the first problem of the
+// input GEMM launch (fc1 + shared up, which read the same x) instead of in a
+// launch of their own: only where that leaves the launch's tiles as they are
+// (the same tile width, the same swap-AB choice at decode sizes).
+bool router_in_input_gemm(const Ctx& c) {
+    const lmoe_config& cf = c.h->cfg;
+    if (route_fp64_all(c)) return false;
+    const int E = cf.num_experts, L = cf.latent, Is = cf.shared_inter;
+    const bool swap2 = c.decode && L % 128 == 0 && Is % 128 == 0;
+    if (swap2) return E % 128 == 0;
+    const int ns2[2] = {L, Is}, ns3[3] = {E, L, Is};
+    return pick_bn(ns3, 3) == pick_bn(ns2, 2);
+}
+
+lmoe_status route_head(Ctx& c, const void* x, bool router_gemm) {
     lmoe_handle* h = c.h;
     const lmoe_config& cf = h->cfg;
     const Plan& p = *c.p;
     char* ws = c.ws;
     LMOE_TRY(cudaMemsetAsync(ws + p.stats, 0, sizeof(WsStats), c.s));
-    if (!route_fp64_all(c)) {
+    if (router_gemm && !route_fp64_all(c)) {
         GemmProblem pr = make_problem(0, p.T, cf.num_experts, EPI_F32, ws + p.logits, cf.num_experts);
         pr.kdim[0] = cf.hidden;
         Operand a[1][2] = {{{x, p.T}, {nullptr, 0}}};
@@ -394,7 +424,7 @@ lmoe_status route_tail(Ctx& c, const void* x, int32_t* idx_out, float* w_out, in
 
 // Routing stages 1-4 in order on the call's stream.
 lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
-    lmoe_status s = route_head(c, x);
+    lmoe_status s = route_head(c, x, true);
     if (s != LMOE_OK) return s;
     return route_tail(c, x, idx_out, w_out, counts_out);
 }
@@ -450,7 +480,7 @@ lmoe_status rerounding(Ctx& c, const void* xa, bool zcheck, bool act_rr);
 // route_head on the call's stream) runs here on the handle's second stream, next
 // to the exact re-roundings of z and a_s, which do not read its outputs; the
 // gather, the first reader of the permutation, waits for it.
-lmoe_status stage_front(Ctx& c, const void* x, void* zdst, const RouteOut& ro) {
+lmoe_status stage_front(Ctx& c, const void* x, void* zdst, const RouteOut& ro, bool with_router) {
     lmoe_handle* h = c.h;
     const lmoe_config& cf = h->cfg;
     const Plan& p = *c.p;
@@ -474,24 +504,34 @@ lmoe_status stage_front(Ctx& c, const void* x, void* zdst, const RouteOut& ro) {
     }
     const bool act_rr = bf16 && h->act_tau > 0.f;
     {
-        GemmProblem pr[2] = {make_problem(0, p.T, L, bf16 && !zcheck ? EPI_BF16 : EPI_F32, ws_c + (zcheck ? p.o : p.z),
-                                          L),
-                             make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is)};
-        pr[0].kdim[0] = H;
-        pr[1].kdim[0] = H;
+        // problems: [router logits (fp32), when merged,] fc1, shared up; all read x
+        GemmProblem pr[3];
+        Operand a[3][2], b[3][2];
+        int np = 0;
+        auto add = [&](GemmProblem q, const void* w, int n) {
+            q.kdim[0] = H;
+            q.a_ptr[0] = xa;
+            q.b_ptr[0] = w;
+            a[np][0] = {xa, p.T};
+            a[np][1] = {nullptr, 0};
+            b[np][0] = {w, n};
+            b[np][1] = {nullptr, 0};
+            pr[np] = q;
+            return np++;
+        };
+        if (with_router) add(make_problem(0, p.T, E, EPI_F32, ws_c + p.logits, E), h->w.router_w, E);
+        const int i_fc1 = add(make_problem(0, p.T, L, bf16 && !zcheck ? EPI_BF16 : EPI_F32,
+                                           ws_c + (zcheck ? p.o : p.z), L),
+                              h->w.fc1_w, L);
+        const int i_su = add(make_problem(0, p.T, Is, bf16 ? EPI_RELU2_BF16 : EPI_RELU2_F32, ws_c + p.as, Is),
+                             h->w.shared_up_w, Is);
         // fc1 in short chunks when z is re-rounded: a smaller fp32 error, a shorter list
-        if (zcheck) pr[0].chunk_kb = LMOE_CHUNK_FC1;
+        if (zcheck) pr[i_fc1].chunk_kb = LMOE_CHUNK_FC1;
         if (act_rr) {
-            set_act_recheck(c, pr[1], &c.st->asflagged);
-            pr[1].chunk_kb = LMOE_CHUNK_SHARED_UP;
+            set_act_recheck(c, pr[i_su], &c.st->asflagged);
+            pr[i_su].chunk_kb = LMOE_CHUNK_SHARED_UP;
         }
-        pr[0].a_ptr[0] = xa;
-        pr[0].b_ptr[0] = h->w.fc1_w;
-        pr[1].a_ptr[0] = xa;
-        pr[1].b_ptr[0] = h->w.shared_up_w;
-        Operand a[2][2] = {{{xa, p.T}, {nullptr, 0}}, {{xa, p.T}, {nullptr, 0}}};
-        Operand b[2][2] = {{{h->w.fc1_w, L}, {nullptr, 0}}, {{h->w.shared_up_w, Is}, {nullptr, 0}}};
-        LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, 2, a, b, xa_f32));
+        LMOE_LAUNCH(gemm_kernels, run_gemm(c, pr, np, a, b, xa_f32));
     }
     // fork: the routing tail on the second stream once the input GEMM is done (the GEMM keeps
     // every SM; the tail's kernels share them with the re-roundings)
@@ -649,10 +689,11 @@ lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y,
     mark(c, 0);
     if (norm_src) LMOE_LAUNCH(1, launch_rmsnorm(norm_src, norm_w, norm_eps, p.T, cf.hidden,
                                                 reinterpret_cast<uint16_t*>(const_cast<void*>(x)), h->num_sms, c.s));
-    s = route_head(c, x);
+    const bool merged = router_in_input_gemm(c);
+    s = route_head(c, x, !merged);
     if (s != LMOE_OK) return s;
     mark(c, 1);
-    s = stage_front(c, x, ws_c + p.zperm, RouteOut{topk_idx, topk_w, expert_counts});
+    s = stage_front(c, x, ws_c + p.zperm, RouteOut{topk_idx, topk_w, expert_counts}, merged);
     if (s != LMOE_OK) return s;
     s = stage_experts(c, ws_c + p.zperm, p.A, reinterpret_cast<const float*>(ws_c + p.wperm), ws_c + p.aperm,
                       reinterpret_cast<float*>(ws_c + p.o), 0);
@@ -909,10 +950,11 @@ lmoe_status latentmoe_ep_front(lmoe_handle* h, const void* x, int T, void* send_
     Ctx c = make_ctx(h, p, ws, stream);
     h->launches = 0;
     mark(c, 0);
-    s = route_head(c, x);
+    const bool merged = router_in_input_gemm(c);
+    s = route_head(c, x, !merged);
     if (s != LMOE_OK) return s;
     mark(c, 1);
-    s = stage_front(c, x, send_rows, RouteOut{nullptr, nullptr, expert_counts});
+    s = stage_front(c, x, send_rows, RouteOut{nullptr, nullptr, expert_counts}, merged);
     if (s != LMOE_OK) return s;
     LMOE_TRY(cudaMemcpyAsync(send_w, c.ws + p.wperm, (size_t)p.A * 4, cudaMemcpyDeviceToDevice, c.s));
     k_publish_error<<<1, 1, 0, c.s>>>(c.err, h->derr);

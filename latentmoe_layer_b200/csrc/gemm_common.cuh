@@ -23,15 +23,16 @@
 namespace lmoe {
 namespace {
 
-constexpr int kMaxMaps = 8;
+constexpr int kMaxMaps = kMaxTensorMaps;
+constexpr int kMaxProb = kMaxProblems;
 constexpr int kGroupM = 16;
 
 struct alignas(64) TcParams {
     CUtensorMap maps[kMaxMaps];
-    GemmProblem prob[2];
+    GemmProblem prob[kMaxProb];
     int nprob;
     int nmaps;
-    int dense_tiles[2];
+    int dense_tiles[kMaxProb];
     DeviceRouting r;
     int* err;
     unsigned spin;
@@ -122,6 +123,19 @@ __device__ __forceinline__ const int4* grouped_records(const DeviceRouting& r) {
 
 __device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) { return pr.n / out_cols; }
 
+// Tiles of the dense problems of a launch, and dense tile t -> its problem
+// (t becomes the tile's index inside that problem).
+__device__ __forceinline__ int dense_total(const TcParams& P) {
+    int n = 0;
+    for (int i = 0; i < P.nprob; ++i) n += P.dense_tiles[i];
+    return n;
+}
+__device__ __forceinline__ int dense_problem(const TcParams& P, int& t) {
+    int p = 0;
+    while (p + 1 < P.nprob && t >= P.dense_tiles[p]) t -= P.dense_tiles[p++];
+    return p;
+}
+
 template <int BN, bool kSwap>
 __device__ __forceinline__ int total_tiles(const TcParams& P) {
     using S = Shape<BN, kSwap>;
@@ -129,7 +143,7 @@ __device__ __forceinline__ int total_tiles(const TcParams& P) {
         const int* pfx = grouped_prefix<S::kActRows>(P.r);
         return pfx[P.r.E] * n_col_tiles(P.prob[0], S::kOutCols);
     }
-    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
+    return dense_total(P);
 }
 
 // Tile t -> coordinates. Dense problems are rasterised in groups of kGroupM
@@ -164,11 +178,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         ti.half = !kSwap && ti.rows <= 64;
         return ti;
     }
-    int p = 0;
-    if (P.nprob > 1 && t >= P.dense_tiles[0]) {
-        t -= P.dense_tiles[0];
-        p = 1;
-    }
+    const int p = dense_problem(P, t);
     const GemmProblem& pr = P.prob[p];
     const int nct = n_col_tiles(pr, S::kOutCols);
     const int mtc = (pr.m_rows + S::kActRows - 1) / S::kActRows;

@@ -285,7 +285,7 @@ struct PairShape {
 
 __device__ __forceinline__ int pair_total_tiles(const TcParams& P) {
     if (P.prob[0].grouped) return P.r.pfx256[P.r.E] * (P.prob[0].n / PairShape::BN);
-    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0);
+    return dense_total(P);
 }
 
 // Pair tile t -> this CTA's half: rows row0 .. row0+rows-1 (rows may be <= 0
@@ -304,10 +304,7 @@ __device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32
         e = pr.expert_mod ? rc.x % pr.expert_mod : rc.x;
         wbase = e * pr.b_rows_per_expert;
     } else {
-        if (P.nprob > 1 && t >= P.dense_tiles[0]) {
-            t -= P.dense_tiles[0];
-            p = 1;
-        }
+        p = dense_problem(P, t);
         const GemmProblem& pr = P.prob[p];
         const int nct = pr.n / PairShape::BN;
         const int mtc = (pr.m_rows + 255) / 256;
@@ -552,6 +549,7 @@ static int dense_tile_count(const GemmProblem& pr) {
 
 cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
                            const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    if (nprob < 1 || nprob > kMaxProb || nmaps > kMaxMaps) return cudaErrorInvalidValue;
     TcParams P;
     fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
     const int sms = tc_num_sms();
@@ -577,6 +575,7 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
 
 cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    if (nprob < 1 || nprob > kMaxProb || nmaps > kMaxMaps) return cudaErrorInvalidValue;
     constexpr int STAGES = 6;
     using S = PairShape;
     constexpr size_t smem = 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 256;
@@ -615,6 +614,7 @@ cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmPr
 
 cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
                                   const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
+    if (nprob < 1 || nprob > kMaxProb || nmaps > kMaxMaps) return cudaErrorInvalidValue;
     TcParams P;
     fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
     int grid = tc_num_sms();

@@ -30,6 +30,8 @@ constexpr int kBM = 128;          // tensor-core tile rows (MMA M)
 constexpr int kBK = 64;           // K elements per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kSimtBM = 64;       // SIMT validation kernels tile rows
 constexpr int kDecodeTN = 32;     // token tile of the swap-AB decode variant (MMA N)
+constexpr int kMaxProblems = 3;   // dense problems in one GEMM launch (router, fc1, shared up)
+constexpr int kMaxTensorMaps = 8; // tensor maps in one GEMM launch
 constexpr float kBandEps = 1e-6f; // tie band of the routing rule
 constexpr int kMaxK = 64;
 constexpr int kMaxE = 1024;

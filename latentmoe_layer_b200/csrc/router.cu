@@ -229,9 +229,13 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // fp64 logits: out[t, e] = sum_h x[t, h] * W_r[e, h]; the bf16 x bf16 (or
 // fp32 x bf16) products are exact in fp64. One work item = one token and a
-// chunk of 64 experts; the token's row is staged in shared memory as fp64 and
-// read as 16-byte vectors (conflict-free), each lane covering 8 consecutive h.
-constexpr int kEChunk = 64;
+// chunk of 16 experts (each warp two of them, their rows streamed together);
+// a block takes a contiguous run of items, so the items of one token follow
+// each other and its row, staged in shared memory as fp64 and read as 16-byte
+// vectors (conflict-free, each lane covering 8 consecutive h), is reused. Small
+// chunks keep a few flagged tokens spread over many SMs.
+constexpr int kERows = 2;                  // experts per warp and pass
+constexpr int kEChunk = 8 * kERows;        // experts per work item (8 warps)
 template <bool kXf32>
 __global__ void __launch_bounds__(256)
     k_logits64(const void* __restrict__ x, const uint16_t* __restrict__ wr, int T, int E, int H,
@@ -239,9 +243,12 @@ __global__ void __launch_bounds__(256)
     extern __shared__ __align__(16) double xrow[];
     const int n = list_count ? *list_count : T;
     const int chunks = (E + kEChunk - 1) / kEChunk;
+    const long long items = (long long)n * chunks;
+    const long long per = (items + gridDim.x - 1) / gridDim.x;
+    const long long i0 = (long long)blockIdx.x * per, i1 = min(items, i0 + per);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int cur = -1;
-    for (long long item = blockIdx.x; item < (long long)n * chunks; item += gridDim.x) {
+    for (long long item = i0; item < i1; ++item) {
         const int li = (int)(item / chunks), ch = (int)(item % chunks);
         const int t = list ? list[li] : li;
         if (!lmoe_check((unsigned)t < (unsigned)T, err)) continue;  // uniform over the block: no barrier skipped unevenly
@@ -259,38 +266,38 @@ __global__ void __launch_bounds__(256)
             __syncthreads();
             cur = t;
         }
-        // each warp: 8 experts of the chunk, 4 rows streamed at once (independent loads)
-        const int e_end = min(E, (ch + 1) * kEChunk);
-        for (int e0 = ch * kEChunk + warp * 8; e0 < min(e_end, ch * kEChunk + warp * 8 + 8); e0 += 4) {
-            const uint16_t* wrow[4];
+        const int e0 = ch * kEChunk + warp * kERows;
+        if (e0 >= E) continue;
+        const uint16_t* wrow[kERows];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) wrow[j] = wr + (size_t)min(e0 + j, E - 1) * H;
-            double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
-            for (int h = lane * 8; h < H; h += 256) {
-                uint4 pk[4];
+        for (int j = 0; j < kERows; ++j) wrow[j] = wr + (size_t)min(e0 + j, E - 1) * H;
+        double acc[kERows][2];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) pk[j] = __ldg(reinterpret_cast<const uint4*>(wrow[j] + h));
-                const double2* xv = reinterpret_cast<const double2*>(xrow + h);
-                double2 xx[4];
+        for (int j = 0; j < kERows; ++j) acc[j][0] = acc[j][1] = 0.0;
+        for (int h = lane * 8; h < H; h += 256) {
+            uint4 pk[kERows];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) xx[q] = xv[q];
+            for (int j = 0; j < kERows; ++j) pk[j] = __ldg(reinterpret_cast<const uint4*>(wrow[j] + h));
+            const double2* xv = reinterpret_cast<const double2*>(xrow + h);
+            double2 xx[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t u[4] = {pk[j].x, pk[j].y, pk[j].z, pk[j].w};
+            for (int q = 0; q < 4; ++q) xx[q] = xv[q];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[j][q & 1] = fma(xx[q].x, (double)__uint_as_float(u[q] << 16), acc[j][q & 1]);
-                        acc[j][q & 1] = fma(xx[q].y, (double)__uint_as_float(u[q] & 0xFFFF0000u), acc[j][q & 1]);
-                    }
+            for (int j = 0; j < kERows; ++j) {
+                const uint32_t u[4] = {pk[j].x, pk[j].y, pk[j].z, pk[j].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[j][q & 1] = fma(xx[q].x, (double)__uint_as_float(u[q] << 16), acc[j][q & 1]);
+                    acc[j][q & 1] = fma(xx[q].y, (double)__uint_as_float(u[q] & 0xFFFF0000u), acc[j][q & 1]);
                 }
             }
+        }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                double a = acc[j][0] + acc[j][1];
+        for (int j = 0; j < kERows; ++j) {
+            double a = acc[j][0] + acc[j][1];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
-                if (lane == 0 && e0 + j < e_end) out[(size_t)t * E + e0 + j] = a;
-            }
+            for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+            if (lane == 0 && e0 + j < E) out[(size_t)t * E + e0 + j] = a;
         }
     }
 }
