@@ -6,12 +6,12 @@
 // band in ascending id, weights = scale * sigma / sum(sigma of the selected).
 //
 // Two precisions of the same decision:
-//  * k_select<float, true>: from fp32 tensor-core logits. The band rule only
+//  * k_select<float, true, .>: from fp32 tensor-core logits. The band rule only
 //    departs from the plain top-k by value when the k-th and (k+1)-th
 //    eligible choice scores are within 1e-6 (or the Gk-th and (Gk+1)-th group
 //    scores are); the token is flagged when either gap is within a margin
 //    `delta` of 1e-6, and flagged tokens are appended to a list.
-//  * k_logits64 + k_select<double, false>: exact-product fp64 logits and the
+//  * k_logits64 + k_select<double, false, .>: exact-product fp64 logits and the
 //    decision in fp64, for the flagged tokens (or for all tokens when x is fp32
 //    or in the fp32 validation mode).
 // If every fp32 choice score is within delta/2 of its fp64 value, an
@@ -43,10 +43,66 @@ __device__ __forceinline__ unsigned first_n_bits(unsigned m, int n) {
     return r;
 }
 
-// Warp-cooperative grouped top-k for one token. c[] and sig[] (length E) live
+// Order-preserving integer keys of choice scores: key(a) > key(b) whenever
+// a > b (-0 sorts just below +0), and every finite score has a key above 0,
+// which marks an ineligible expert.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ unsigned long long order_key(double v) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    return (u >> 63) ? ~u : (u | (1ull << 63));
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ double key_value(unsigned long long k) {
+    return __longlong_as_double((long long)((k >> 63) ? (k & ~(1ull << 63)) : ~k));
+}
+
+// tau = the k-th largest eligible choice score and next = the (k+1)-th (-inf
+// when fewer than k+1 are eligible), equal scores counted once each, as k
+// rounds of taking the largest would. Bisection on the keys: bit b of tau's key
+// (from the top) is set when at least k eligible keys are >= the prefix with
+// that bit set; one compare per element and one warp sum per bit. Lane l holds
+// the keys of experts l + 32 i, i < kNI (bit i of elig: eligible).
+template <typename F, int kNI>
+__device__ __forceinline__ void kth_and_next(const F* c, unsigned elig, int nI, int k, F& tau, F& next) {
+    using U = decltype(order_key(F(0)));
+    const int lane = threadIdx.x & 31;
+    U key[kNI];
+#pragma unroll
+    for (int i = 0; i < kNI; ++i) key[i] = (i < nI && ((elig >> i) & 1u)) ? order_key(c[lane + (i << 5)]) : (U)0;
+    U res = 0;
+    for (int b = 8 * (int)sizeof(U) - 1; b >= 0; --b) {
+        const U cand = res | ((U)1 << b);
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < kNI; ++i) cnt += key[i] >= cand ? 1 : 0;
+        if (__reduce_add_sync(0xFFFFFFFFu, cnt) >= k) res = cand;
+    }
+    int at_or_above = 0;
+    U below = 0;
+#pragma unroll
+    for (int i = 0; i < kNI; ++i) {
+        at_or_above += key[i] >= res ? 1 : 0;
+        if (key[i] < res && key[i] > below) below = key[i];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const U o = __shfl_xor_sync(0xFFFFFFFFu, below, off);
+        below = o > below ? o : below;
+    }
+    tau = key_value(res);
+    if (__reduce_add_sync(0xFFFFFFFFu, at_or_above) > k) next = tau;
+    else next = below == 0 ? -(F)INFINITY : key_value(below);
+}
+
+// Warp-cooperative grouped top-k for one token.// Warp-cooperative grouped top-k for one token. c[] and sig[] (length E) live
 // in this warp's shared memory. Writes idx (ascending) and weights; returns
 // true when the token must be re-decided in fp64 (kFlag only).
-template <typename F, bool kFlag>
+template <typename F, bool kFlag, int kNI>
 __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int k, float scale, F delta,
                             int32_t* idx_out, float* w_out) {
     const int lane = threadIdx.x & 31;
@@ -134,35 +190,9 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
         const int e = lane + (i << 5);
         if (e < E && ((keep >> (e / per)) & 1u)) elig |= 1u << i;
     }
-    // tau = k-th largest eligible choice score (k rounds of warp argmax).
-    unsigned removed = 0;
-    F tau = ninf, next = ninf;
-    for (int j = 0; j < (kFlag ? k + 1 : k); ++j) {
-        F best = ninf;
-        int be = 0x7FFFFFFF;
-        for (int i = 0; i < nI; ++i) {
-            const int e = lane + (i << 5);
-            if (((elig & ~removed) >> i) & 1u) {
-                F v = c[e];
-                if (v > best) {
-                    best = v;
-                    be = e;
-                }
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            F ob = __shfl_xor_sync(0xFFFFFFFFu, best, off);
-            int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-            if (ob > best || (ob == best && oe < be)) {
-                best = ob;
-                be = oe;
-            }
-        }
-        if (be != 0x7FFFFFFF && (be & 31) == lane) removed |= 1u << (be >> 5);
-        if (j < k) tau = best;
-        else next = best;  // (k+1)-th largest eligible score, -inf if there is none
-    }
+    // tau = k-th largest eligible choice score, next = the (k+1)-th
+    F tau, next;
+    kth_and_next<F, kNI>(c, elig, nI, k, tau, next);
     if (kFlag) flag |= (tau - next) <= eps + delta;
     // A = {c > tau + eps}; the band |c - tau| <= eps fills the rest in ascending id.
     int nA = 0;
@@ -196,7 +226,7 @@ __device__ bool warp_select(const F* c, const F* sig, int E, int G, int Gk, int 
     return flag;
 }
 
-template <typename F, bool kFlag>
+template <typename F, bool kFlag, int kNI>
 __global__ void __launch_bounds__(kWarps * 32)
     k_select(const F* __restrict__ logits, const float* __restrict__ bias, int T, int E, int G, int Gk, int k,
              float scale, float delta, const int* __restrict__ list, const int* __restrict__ list_count,
@@ -217,8 +247,8 @@ __global__ void __launch_bounds__(kWarps * 32)
             c[e] = s + (F)bias[e];
         }
         __syncwarp();
-        bool flag = warp_select<F, kFlag>(c, sig, E, G, Gk, k, scale, (F)delta, idx + (size_t)t * k,
-                                          wgt + (size_t)t * k);
+        bool flag = warp_select<F, kFlag, kNI>(c, sig, E, G, Gk, k, scale, (F)delta, idx + (size_t)t * k,
+                                               wgt + (size_t)t * k);
         if (kFlag && flag && lane == 0) {
             int pos = atomicAdd(flag_count, 1);
             flaglist[pos] = t;
@@ -311,7 +341,13 @@ cudaError_t launch_router_select(const lmoe_handle* h, const Plan& p, char* ws, 
     if (blocks > 4 * h->num_sms) blocks = 4 * h->num_sms;
     size_t smem = (size_t)kWarps * 2 * E * sizeof(float);
     WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
-    k_select<float, true><<<blocks, kWarps * 32, smem, s>>>(
+    // keys per lane: E / 32 rounded up to 16 or 32 (E <= kMaxE = 1024)
+    auto kern = E <= 512 ? k_select<float, true, 16> : k_select<float, true, 32>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<blocks, kWarps * 32, smem, s>>>(
         reinterpret_cast<const float*>(ws + p.logits), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
         c.routed_scaling_factor, h->flag_delta, nullptr, nullptr, reinterpret_cast<int32_t*>(ws + p.idx),
         reinterpret_cast<float*>(ws + p.wgt), reinterpret_cast<int*>(ws + p.flaglist), &st->flagged, &st->device_error);
@@ -349,15 +385,15 @@ cudaError_t launch_router_select64(const lmoe_handle* h, const Plan& p, char* ws
     WsStats* st = reinterpret_cast<WsStats*>(ws + p.stats);
     int E = c.num_experts;
     size_t smem = (size_t)kWarps * 2 * E * sizeof(double);
+    auto kern = E <= 512 ? k_select<double, false, 16> : k_select<double, false, 32>;
     if (smem > 48 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_select<double, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     int blocks = all ? (p.T + kWarps - 1) / kWarps : h->num_sms;
     if (blocks > 4 * h->num_sms) blocks = 4 * h->num_sms;
     if (blocks < 1) blocks = 1;
-    k_select<double, false><<<blocks, kWarps * 32, smem, s>>>(
+    kern<<<blocks, kWarps * 32, smem, s>>>(
         reinterpret_cast<const double*>(ws + p.logits64), h->w.e_bias, p.T, E, c.n_group, c.topk_group, c.top_k,
         c.routed_scaling_factor, 0.f, all ? nullptr : reinterpret_cast<const int*>(ws + p.flaglist),
         all ? nullptr : &st->flagged, reinterpret_cast<int32_t*>(ws + p.idx), reinterpret_cast<float*>(ws + p.wgt),

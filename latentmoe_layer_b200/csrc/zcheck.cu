@@ -25,6 +25,7 @@
 // threshold whose fp32 value lies within the accumulation-error margin of a
 // midpoint, and k_recheck<relu2> recomputes them the same way.
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <stdint.h>
 
 #include "lmoe_internal.h"
@@ -78,6 +79,7 @@ template <typename LoadA>
 __device__ __forceinline__ void dot_pairs(LoadA load_a, const uint4* __restrict__ wr, int K8, int lane, float& hi,
                                           float& lo) {
     float h[4] = {0.f, 0.f, 0.f, 0.f}, l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int k = lane; k < K8; k += 32) {
         const uint4 a = load_a(k), b = __ldg(wr + k);
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -185,29 +187,31 @@ __global__ void __launch_bounds__(256) k_round_flag(const float* __restrict__ z3
     }
 }
 
-// Exact re-rounding of the listed z elements, one CTA per segment of rowtab: the
-// segment's row of x (K bf16, K a multiple of 8) is staged once in shared
-// memory, and each warp takes one listed element at a time, streaming its row
-// of W (fc1_latent_proj, resident in L2 across the launch). The sum is the
-// error-free double-fp32 sum of k_recheck.
+// Exact re-rounding of the listed z elements, `split` CTAs per segment of
+// rowtab (more than one when there are few rows, so the entries spread over
+// the SMs): the segment's row of x (K bf16, K a multiple of 8) is staged in
+// shared memory, and each warp takes one listed element at a time, streaming
+// its row of W (fc1_latent_proj, resident in L2 across the launch). The sum is
+// the error-free double-fp32 sum of k_recheck.
 __global__ void __launch_bounds__(256) k_recheck_rows(const uint16_t* __restrict__ A, int a_rows,
                                                       const uint16_t* __restrict__ W, int w_rows, int K, int* err,
                                                       const int2* __restrict__ list, int cap,
                                                       const int4* __restrict__ rowtab, const int* __restrict__ nrowtab,
-                                                      uint16_t* __restrict__ out, int ldo) {
+                                                      uint16_t* __restrict__ out, int ldo, int split) {
     extern __shared__ uint4 xs[];  // K / 8 vectors
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int K8 = K / 8;
-    const int n = *nrowtab;
-    for (int item = blockIdx.x; item < n; item += gridDim.x) {
-        const int4 rt = rowtab[item];
+    const long long n = (long long)*nrowtab * split;
+    for (long long item = blockIdx.x; item < n; item += gridDim.x) {
+        const int part = (int)(item % split);  // this CTA's share of the segment's entries
+        const int4 rt = rowtab[item / split];
         if (!lmoe_check((unsigned)rt.x < (unsigned)a_rows, err)) continue;  // uniform over the CTA
         __syncthreads();
         const uint4* xr = reinterpret_cast<const uint4*>(A + (size_t)rt.x * K);
         for (int k = threadIdx.x; k < K8; k += blockDim.x) xs[k] = __ldg(xr + k);
         __syncthreads();
         const int e1 = min(rt.y + rt.z, cap);
-        for (int e = rt.y + warp; e < e1; e += nw) {
+        for (int e = rt.y + part * nw + warp; e < e1; e += nw * split) {
             const int2 ent = list[e];
             if (!lmoe_check((unsigned)ent.y < (unsigned)w_rows, err)) continue;
             const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)ent.y * K);
@@ -281,7 +285,11 @@ cudaError_t launch_recheck_rows(const uint16_t* A, int a_rows, const uint16_t* W
         cudaError_t e = cudaFuncSetAttribute(k_recheck_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_recheck_rows<<<sms * 4, 256, smem, s>>>(A, a_rows, W, w_rows, K, err, list, cap, rowtab, nrowtab, out, ldo);
+    // rows (segments) below four CTAs per SM: split each segment's entries over up to 8 CTAs
+    const long long segs = (long long)a_rows * ((w_rows + kSegCols - 1) / kSegCols);
+    const int split = (int)std::max<long long>(1, std::min<long long>(8, (long long)sms * 4 / std::max(segs, 1LL)));
+    k_recheck_rows<<<sms * 4, 256, smem, s>>>(A, a_rows, W, w_rows, K, err, list, cap, rowtab, nrowtab, out, ldo,
+                                              split);
     return cudaGetLastError();
 }
 
