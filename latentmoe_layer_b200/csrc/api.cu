@@ -181,6 +181,20 @@ int pick_bn(const int* ns, int cnt) {
     return 0;
 }
 
+// Tokens per tile of a swap-AB (decode) launch: 64 where every problem is dense
+// with at most 64 rows and 64-token tiles take fewer waves over the SMs than
+// 32-token ones (each wave streams the same weight tiles; more tiles in a wave
+// keep more SMs streaming), else kDecodeTN.
+int decode_bn(const GemmProblem* probs, int nprob, int sms) {
+    long long t32 = 0, t64 = 0;
+    for (int i = 0; i < nprob; ++i) {
+        if (probs[i].grouped || probs[i].m_rows > 64) return kDecodeTN;
+        t32 += (long long)((probs[i].m_rows + kDecodeTN - 1) / kDecodeTN) * (probs[i].n / 128);
+        t64 += probs[i].n / 128;
+    }
+    return (t64 + sms - 1) / sms < (t32 + sms - 1) / sms ? 64 : kDecodeTN;
+}
+
 struct Ctx {
     lmoe_handle* h;
     const Plan* p;
@@ -212,7 +226,7 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
         ns[i] = probs[i].n;
         swap = swap && probs[i].n % 128 == 0;
     }
-    const int bn = swap ? kDecodeTN : pick_bn(ns, nprob);
+    const int bn = swap ? decode_bn(probs, nprob, c.h->num_sms) : pick_bn(ns, nprob);
     if (bn == 0) return cudaErrorInvalidValue;
     // 256 x 256 tiles on 2-SM pairs (option 4): each CTA of the pair loads 128 rows of B
     const bool pair = !swap && bn == 256 && c.h->gemm_path == 4;
@@ -229,7 +243,7 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
                     am = probs[j].a_map[0];
             if (am < 0) {
                 if (nm >= kMaxTensorMaps ||
-                    !encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? kDecodeTN : kBM))
+                    !encode_bf16(&maps[nm], a[i][sg].ptr, a[i][sg].rows, K, swap ? bn : kBM))
                     return cudaErrorInvalidValue;
                 am = nm++;
             }
@@ -250,7 +264,7 @@ cudaError_t run_gemm(Ctx& c, GemmProblem* probs, int nprob, const Operand (*a)[2
         }
         probs[i].out_map = nm++;
     }
-    if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
+    if (swap) return launch_gemm_tc_decode(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
     if (pair) return launch_gemm_tc_pair(maps, nm, probs, nprob, c.r, c.err, c.h->spin_limit, c.s);
     return launch_gemm_tc(maps, nm, probs, nprob, bn, c.r, c.err, c.h->spin_limit, c.s);
 }

@@ -125,15 +125,16 @@ __device__ __forceinline__ int n_col_tiles(const GemmProblem& pr, int out_cols) 
 
 // Tiles of the dense problems of a launch, and dense tile t -> its problem
 // (t becomes the tile's index inside that problem).
+static_assert(kMaxProb == 3, "dense_total / dense_problem are written out for three problems");
 __device__ __forceinline__ int dense_total(const TcParams& P) {
-    int n = 0;
-    for (int i = 0; i < P.nprob; ++i) n += P.dense_tiles[i];
-    return n;
+    return P.dense_tiles[0] + (P.nprob > 1 ? P.dense_tiles[1] : 0) + (P.nprob > 2 ? P.dense_tiles[2] : 0);
 }
 __device__ __forceinline__ int dense_problem(const TcParams& P, int& t) {
-    int p = 0;
-    while (p + 1 < P.nprob && t >= P.dense_tiles[p]) t -= P.dense_tiles[p++];
-    return p;
+    if (P.nprob < 2 || t < P.dense_tiles[0]) return 0;
+    t -= P.dense_tiles[0];
+    if (P.nprob < 3 || t < P.dense_tiles[1]) return 1;
+    t -= P.dense_tiles[1];
+    return 2;
 }
 
 template <int BN, bool kSwap>

@@ -612,21 +612,24 @@ cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmPr
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
                                   const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s) {
     if (nprob < 1 || nprob > kMaxProb || nmaps > kMaxMaps) return cudaErrorInvalidValue;
+    if (bn != kDecodeTN && (bn != 64 || probs[0].grouped)) return cudaErrorInvalidValue;
     TcParams P;
     fill_params(P, maps, nmaps, probs, nprob, r, err, spin_limit);
     int grid = tc_num_sms();
     if (!probs[0].grouped) {
         long long tiles = 0;
         for (int i = 0; i < nprob; ++i) {
-            P.dense_tiles[i] = dense_tile_count<kDecodeTN, true>(probs[i]);
+            P.dense_tiles[i] = bn == 64 ? dense_tile_count<64, true>(probs[i]) : dense_tile_count<kDecodeTN, true>(probs[i]);
             tiles += P.dense_tiles[i];
         }
         if (tiles < grid) grid = (int)tiles;
         if (grid < 1) return cudaSuccess;
     }
+    // 64-token tiles: every token of a short batch in one tile, one pass over each weight tile
+    if (bn == 64) return launch_impl<64, 8, true>(P, grid, s);
     return launch_impl<kDecodeTN, 10, true>(P, grid, s);
 }
 

@@ -182,7 +182,8 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
                            const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
 cudaError_t launch_gemm_tc_pair(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
                                 const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
-cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob,
+// bn: tokens per tile, kDecodeTN or (dense problems of at most 64 rows) 64.
+cudaError_t launch_gemm_tc_decode(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
                                   const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
 cudaError_t launch_gemm_tc_nvfp4(const CUtensorMap* maps, int nmaps, const GemmProblem* probs, int nprob, int bn,
                                  const DeviceRouting& r, int* err, unsigned spin_limit, cudaStream_t s);
