@@ -200,6 +200,43 @@ def test_token_permutation_equivariance_bitwise():
     assert torch.equal(yp, y[perm])
 
 
+@pytest.mark.parametrize("shape", [NANO_DECODE, RAGGED])
+def test_forward_replays_from_a_cuda_graph(shape):
+    """A forward captured into a CUDA graph (the routing tail on the handle's second stream is
+    forked from and joined back into the captured stream) replays bit for bit like eager calls,
+    also after new data is written into the captured x. Nano: router logits inside the input GEMM
+    launch; ragged: their own launch."""
+    import torch
+    layer, dev = H.device_layer(shape)
+    x = dev["x"].clone()
+    y = torch.empty((shape.T, shape.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    layer.forward(x, y, idx=idx)  # allocates the workspace outside the capture
+    torch.cuda.synchronize()
+    y_eager, idx_eager = y.clone(), idx.clone()
+    x2 = torch.roll(dev["x"], 1, dims=0).contiguous()
+    layer.forward(x2, y, idx=idx)
+    torch.cuda.synchronize()
+    y2_eager, idx2_eager = y.clone(), idx.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            layer.forward(x, y, idx=idx)
+    torch.cuda.current_stream().wait_stream(s)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager) and torch.equal(idx, idx_eager)
+    x.copy_(x2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2_eager) and torch.equal(idx, idx2_eager)
+    assert layer.stats().device_error == 0
+    del g
+
+
 def test_route_entry_point_matches_forward():
     import torch
     layer, dev = H.device_layer(RAGGED)
