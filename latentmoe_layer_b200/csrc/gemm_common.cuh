@@ -42,7 +42,9 @@ struct TileInfo {
     int p;       // problem
     int row0;    // first activation row (permuted row for grouped problems)
     int rows;    // valid activation rows in this tile
-    int wrow0;   // first weight row (row of B)
+    int wrow0;   // first weight row this CTA loads (row of B)
+    int wcol0;   // weight row of the tile's first output column (differs from wrow0 in the second
+                 // CTA of a 2-SM pair, which loads the upper half of the pair's B rows)
     int col0;    // first output column
     int e;       // expert of a grouped tile (-1 for dense problems)
     bool half;   // non-swapped tile with <= 64 valid rows: M = 64 MMAs (the expert's ragged tail)
@@ -72,7 +74,7 @@ __device__ __forceinline__ void rr_append_warp(const GemmProblem& pr, int n, con
             const int i = w * 32 + __ffs(m) - 1;
             m &= m - 1u;
             const int r = swap ? c0 + i : lane_row, col = swap ? lane_row : c0 + i;
-            if (pos < pr.rr_cap) pr.rr_list[pos] = make_int2(ti.row0 + r, ti.wrow0 + col);
+            if (pos < pr.rr_cap) pr.rr_list[pos] = make_int2(ti.row0 + r, ti.wcol0 + col);
             ++pos;
         }
     }
@@ -175,6 +177,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
         ti.rows = rc.z;
         ti.col0 = ct * S::kOutCols;
         ti.wrow0 = e * pr.b_rows_per_expert + ti.col0;
+        ti.wcol0 = ti.wrow0;
         ti.e = e;
         ti.half = !kSwap && ti.rows <= 64;
         return ti;
@@ -198,6 +201,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int t) {
     ti.rows = min(S::kActRows, pr.m_rows - ti.row0);
     ti.col0 = ct * S::kOutCols;
     ti.wrow0 = ti.col0;
+    ti.wcol0 = ti.col0;
     ti.e = -1;
     ti.half = !kSwap && ti.rows <= 64;
     return ti;

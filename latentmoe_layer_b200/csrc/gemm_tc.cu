@@ -320,7 +320,8 @@ __device__ __forceinline__ TileInfo pair_decode(const TcParams& P, int t, uint32
     ti.row0 = prow0 + (int)rank * 128;
     ti.rows = min(128, prows - (int)rank * 128);
     ti.col0 = ct * PairShape::BN;
-    ti.wrow0 = wbase + ti.col0 + (int)rank * 128;
+    ti.wrow0 = wbase + ti.col0 + (int)rank * 128;  // this CTA's half of the pair's B rows
+    ti.wcol0 = wbase + ti.col0;                      // the output columns span both halves
     ti.e = e;
     ti.half = false;
     return ti;

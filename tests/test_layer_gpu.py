@@ -21,6 +21,8 @@ GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE, GEMM_SIMT, GEMM_PREFILL_PAIR = range(5)
 # several tiles and ragged tails in every dimension the kernels tile
 RAGGED = LayerShape("ragged", T=333, H=512, L=256, E=64, k=6, G=4, Gk=2, I=384, Is=640)
 RAGGED_X32 = replace(RAGGED, name="ragged_x32", x_f32=True, T=97)
+# every GEMM width a multiple of 256, so that option 4 runs 2-SM pair tiles (RAGGED's widths do not)
+PAIRW = LayerShape("pair_widths", T=600, H=1024, L=512, E=64, k=4, G=4, Gk=2, I=768, Is=1024)
 
 
 def run_and_compare(shape, mode=0, path=GEMM_AUTO, full=True):
@@ -58,6 +60,11 @@ def test_tiny_fp32_validation_mode():
 @pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_PREFILL_PAIR, GEMM_DECODE, GEMM_SIMT])
 def test_ragged_bf16(path):
     run_and_compare(RAGGED, mode=0, path=path)
+
+
+@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_PREFILL_PAIR, GEMM_DECODE])
+def test_pair_widths_bf16(path):
+    run_and_compare(PAIRW, mode=0, path=path)
 
 
 def test_ragged_fp32_x_bf16_mode():
@@ -431,6 +438,48 @@ def test_activations_above_tau_are_exact_roundings():
           (above, flips_below, below, int(big_s.sum()), int((got_s[~big_s] != ref_s[~big_s]).sum()),
            int((~big_s).sum()), st.ae_rechecked, st.as_rechecked))
     assert above > 0 and big_s.any() and st.ae_rechecked > 0 and st.as_rechecked > 0
+
+
+@pytest.mark.parametrize("path", [GEMM_PREFILL, GEMM_PREFILL_PAIR, GEMM_DECODE])
+def test_activation_rerounding_exact_on_every_gemm_path(path):
+    """With tau lowered to 0.25, so that a share of the activations at this width is listed, every
+    expert and shared-expert activation with h > tau equals the exact rounding on each GEMM path, all
+    rows: single-CTA tiles, 2-SM pair tiles (whose second CTA loads the upper half of the tile's weight
+    rows while its outputs span the whole tile) and the swap-AB decode tiles."""
+    import torch
+    shape = PAIRW
+    layer, dev = H.device_layer(shape)
+    layer.set_option(0, path)
+    layer.set_option(lm_opt("OPT_ACT_RECHECK_TAU"), 250)
+    tau = 0.25
+    T, L, I, Is, A = shape.T, shape.L, shape.I, shape.Is, shape.T * shape.k
+    y = torch.empty((T, shape.H), dtype=torch.float32, device="cuda")
+    layer.forward(dev["x"], y)
+    torch.cuda.synchronize()
+    st = layer.stats()
+    assert st.device_error == 0 and st.ae_rechecked > 0 and st.as_rechecked > 0
+    lay = layer.layout(T)
+    offs = layer.ws_view(lay.offsets, (shape.E + 1,), torch.int32).cpu().numpy()
+    perm = layer.ws_view(lay.perm, (A,), torch.int32)
+    zb = layer.ws_view(lay.z, (T, L), torch.bfloat16)
+    ae = layer.ws_view(lay.act_e, (A, I), torch.bfloat16)
+    asb = layer.ws_view(lay.act_s, (T, Is), torch.bfloat16)
+    above = 0
+    for e in range(shape.E):
+        if offs[e + 1] == offs[e]:
+            continue
+        rt = torch.arange(int(offs[e]), int(offs[e + 1]), device="cuda")
+        h, ref = _exact_relu2((L, I), H.bf16_to_bits(zb[perm[rt].long()]), H.bf16_to_bits(dev["up_w"][e]))
+        got = H.bf16_to_bits(ae[rt])
+        big = h > tau
+        above += int(big.sum())
+        assert np.array_equal(got[big], ref[big]), "path %d expert %d: a_e above tau differs" % (path, e)
+    hs, ref_s = _exact_relu2((shape.H, Is), H.host_x(shape, dev, np.arange(T)), H.bf16_to_bits(dev["shared_up_w"]))
+    got_s = H.bf16_to_bits(asb)
+    big_s = hs > tau
+    assert np.array_equal(got_s[big_s], ref_s[big_s]), "path %d: a_s above tau differs" % path
+    print("path %d: a_e %d above tau exact (%d listed), a_s %d above tau exact (%d listed)" %
+          (path, above, st.ae_rechecked, int(big_s.sum()), st.as_rechecked))
 
 
 # ---------------------------------------------------------------- ties
