@@ -18,9 +18,10 @@ assert os.environ.get("LATENTMOE_CHECKS") == "1" and lm.LIB_PATH.endswith("libla
 
 
 def case_layer():
-    from test_layer_gpu import run_and_compare, RAGGED, RAGGED_X32, TINY
+    from test_layer_gpu import run_and_compare, RAGGED, RAGGED_X32, TINY, PAIRW
+    # PAIRW: widths that make option 4 run 2-SM pair tiles (RAGGED's do not)
     for shape, mode, path in ((TINY, 0, 1), (RAGGED, 0, 1), (RAGGED, 0, 2), (RAGGED, 0, 3), (RAGGED, 0, 4),
-                              (RAGGED_X32, 0, 1), (RAGGED, 1, 0)):
+                              (PAIRW, 0, 4), (RAGGED_X32, 0, 1), (RAGGED, 1, 0)):
         (ma, rf), layer = run_and_compare(shape, mode=mode, path=path)
         assert layer.stats().device_error == 0
         print("%s mode=%d path=%d max_abs=%.3g rel_fro=%.3g" % (shape.name, mode, path, ma, rf))
