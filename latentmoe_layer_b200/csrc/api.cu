@@ -1,16 +1,25 @@
-// api.cpp -- the C ABI of the LatentMoE layer forward (include/latentmoe.h):
+// api.cu -- the C ABI of the LatentMoE layer forward (include/latentmoe.h):
 // argument validation, workspace carving, TMA descriptor encoding and the
-// launch sequence. Every launch goes to the caller's stream; nothing here
-// synchronises except the diagnostic entry points that say so.
+// launch sequence. Every launch goes to the caller's stream or to the handle's
+// second stream, forked from and joined back into the caller's stream within
+// the call; nothing here synchronises except the diagnostic entry points that
+// say so.
 //
 // Launch sequence of latentmoe_forward (bf16 mode):
-//   1 router GEMM       logits = x W_r^T (fp32, tensor cores)
+//   1 input GEMM        logits = x W_r^T (fp32), z = x W_fc1^T (fp32 when z is
+//                       re-rounded) and a_s = relu2(x W_su^T) (bf16): one launch,
+//                       three problems (the router in a launch of its own where
+//                       the tile shapes differ)
+//   -- fork: on the second stream, steps 2-4; on the caller's stream, step 5
 //   2 select            sigmoid, +bias, grouped top-k, weights; near-edge flags
 //   3 fp64 re-check     flagged tokens: exact-product fp64 logits and decision
 //   4 permutation       counts, offsets, tile prefixes, perm, slot, row weights
-//   5 input GEMM        z = x W_fc1^T (bf16) and a_s = relu2(x W_su^T) (bf16)
+//   5 exact re-rounding z = bf16 of the exact sum for the elements near a
+//                       rounding midpoint; the same for the large a_s
+//   -- join
 //   6 gather            z rows into expert order
-//   7 expert up GEMM    a = relu2(z_e W_up[e]^T) (bf16), grouped by expert
+//   7 expert up GEMM    a = relu2(z_e W_up[e]^T) (bf16), grouped by expert,
+//                       then the exact re-rounding of its large activations
 //   8 expert down GEMM  o = w * (a_e W_down[e]^T) (fp32), grouped by expert
 //   9 combine           comb[t] = bf16(sum over the token's k rows, ascending id)
 //  10 output GEMM       y = comb W_fc2^T + a_s W_sd^T (fp32), one K-concatenated GEMM
@@ -436,7 +445,8 @@ lmoe_status route_tail(Ctx& c, const void* x, int32_t* idx_out, float* w_out, in
     return LMOE_OK;
 }
 
-// Routing stages 1-4 in order on the call's stream.
+// Routing in order on the call's stream (latentmoe_route): the router GEMM,
+// then steps 2-4 of the file comment.
 lmoe_status do_route(Ctx& c, const void* x, int32_t* idx_out, float* w_out, int32_t* counts_out) {
     lmoe_status s = route_head(c, x, true);
     if (s != LMOE_OK) return s;
@@ -483,17 +493,17 @@ __global__ void k_publish_error(const int* derr, int* herr) {
     if (v != 0) *(volatile int*)herr = v;
 }
 
-// The layer on x (launches 1-10 of the file comment). With `resid` (bf16
-// [T, H]) the output GEMM adds it: y = resid + layer(x).
+// Experts whose weights the handle holds (a shard of them for expert parallelism).
 int experts_held(const lmoe_config& c) { return c.local_experts > 0 ? c.local_experts : c.num_experts; }
 
 lmoe_status rerounding(Ctx& c, const void* xa, bool zcheck, bool act_rr);
 
-// Steps 5-6: z = x W_fc1^T and a_s = relu2(x W_su^T) (one launch), then the
-// rows of z in expert order into zdst. The routing tail (route_tail, after
-// route_head on the call's stream) runs here on the handle's second stream, next
-// to the exact re-roundings of z and a_s, which do not read its outputs; the
-// gather, the first reader of the permutation, waits for it.
+// Steps 1-6 of the file comment: the input GEMM (z = x W_fc1^T and
+// a_s = relu2(x W_su^T), with the router logits as a first problem when
+// with_router), then the rows of z in expert order into zdst. The routing tail
+// (route_tail, after route_head on the call's stream) runs here on the handle's
+// second stream, next to the exact re-roundings of z and a_s, which do not read
+// its outputs; the gather, the first reader of the permutation, waits for it.
 lmoe_status stage_front(Ctx& c, const void* x, void* zdst, const RouteOut& ro, bool with_router) {
     lmoe_handle* h = c.h;
     const lmoe_config& cf = h->cfg;
@@ -692,6 +702,9 @@ lmoe_status stage_back(Ctx& c, const float* o, float* y, const uint16_t* resid) 
     return LMOE_OK;
 }
 
+// The layer on x (steps 1-10 of the file comment). With norm_src the pre-norm
+// runs first and x is its output; with `resid` (bf16 [T, H]) the output GEMM
+// adds it: y = resid + layer(x).
 lmoe_status forward_impl(lmoe_handle* h, const Plan& p, const void* x, float* y, void* ws, void* stream,
                          int32_t* topk_idx, float* topk_w, int32_t* expert_counts, const uint16_t* resid,
                          const uint16_t* norm_src, const uint16_t* norm_w, double norm_eps) {
