@@ -29,7 +29,8 @@
  * activations are rounded to bf16 as GEMM operands; z, which every routed
  * expert of a token reads, is re-rounded so that it equals the exact rounding
  * of x W_fc1^T whenever the fp32 error of an element is below the margin of
- * LMOE_OPT_Z_RECHECK_DELTA);
+ * LMOE_OPT_Z_RECHECK_DELTA, and the expert and shared-expert activations with
+ * h above LMOE_OPT_ACT_RECHECK_TAU likewise);
  * LMOE_MODE_FP32 is a validation mode with fp32 operands and no intermediate
  * rounding.
  *
@@ -40,6 +41,17 @@
  * host-visible memory and return; the call that launched it, or the next call
  * on the handle, returns LMOE_ERR_TIMEOUT. Launch failures return
  * LMOE_ERR_CUDA. T = 0 returns LMOE_OK and launches nothing.
+ *
+ * Streams: calls are asynchronous on the caller's stream. latentmoe_forward,
+ * latentmoe_forward_block and latentmoe_ep_front also use a second stream the
+ * handle owns (created by latentmoe_create on the device current then): within
+ * the call the routing kernels are forked onto it after the input GEMM and
+ * joined back into the caller's stream before the first kernel that reads
+ * their outputs, so work enqueued afterwards on the caller's stream sees the
+ * call complete. These calls can be captured into a CUDA graph. A handle's
+ * calls must not be issued from several host threads at once; calls from one
+ * thread on different streams are correct, and their routing kernels run in
+ * turn on the handle's stream.
  *
  * Determinism: the same inputs give bitwise-identical outputs (no floating-
  * point atomics; sums run in a fixed order).
