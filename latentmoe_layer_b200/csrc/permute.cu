@@ -227,9 +227,9 @@ __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ src, i
 #pragma unroll
             for (int j = 0; j < 8; ++j) v[j] = ld_global_nc_v4(s + c + 32 * j);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) st_global_v4(d + c + 32 * j, v[j]);
+            for (int j = 0; j < 8; ++j) st_global_cs_v4(d + c + 32 * j, v[j]);  // rows far beyond L2
         }
-        for (; c < vec_per_row; c += 32) st_global_v4(d + c, ld_global_nc_v4(s + c));
+        for (; c < vec_per_row; c += 32) st_global_cs_v4(d + c, ld_global_nc_v4(s + c));
     }
 }
 
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(256)
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < k; ++j) {
                 if (!lmoe_check((unsigned)sl[j] < (unsigned)o_rows, err)) continue;
-                float4 v = __ldg(&o[(size_t)sl[j] * L4 + c]);
+                float4 v = __ldcs(&o[(size_t)sl[j] * L4 + c]);  // o is read once: evict first
                 acc.x += v.x;
                 acc.y += v.y;
                 acc.z += v.z;

@@ -78,8 +78,10 @@ __device__ __forceinline__ uint4 ld_global_nc_v4(const uint4* p) {
                  : "l"(p));
     return v;
 }
-__device__ __forceinline__ void st_global_v4(uint4* p, uint4 v) {
-    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+// Streaming (evict-first) store: for data far larger than L2 that is written
+// once and read back later by another kernel.
+__device__ __forceinline__ void st_global_cs_v4(uint4* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 
