@@ -67,6 +67,17 @@ def test_pair_widths_bf16(path):
     run_and_compare(PAIRW, mode=0, path=path)
 
 
+# T = 40 at decode sizes: the input GEMM (router merged, (128 + 2048 + 8192) / 128 = 81 weight tiles)
+# runs one wave of 64-token tiles, each holding 40 valid tokens, instead of two waves of 32-token tiles
+DEC64 = LayerShape("decode_64_tiles", T=40, H=1024, L=2048, E=128, k=4, G=4, Gk=2, I=512, Is=8192)
+
+
+def test_decode_64_token_tiles_with_a_partial_tile():
+    (ma, rf), layer = run_and_compare(DEC64, mode=0, path=GEMM_AUTO)
+    assert layer.stats().device_error == 0
+    print("decode_64_tiles max_abs=%.3g rel_fro=%.3g" % (ma, rf))
+
+
 def test_ragged_fp32_x_bf16_mode():
     run_and_compare(RAGGED_X32, mode=0, path=GEMM_PREFILL)
 
