@@ -41,10 +41,17 @@
 namespace lmoe {
 namespace {
 
-template <int BN, int STAGES, bool kSwap>
+// CG: shared-memory stages released per MMA commit. A tcgen05.commit holds the
+// tensor pipe for about an MMA's latency (~230 cycles measured, against 130 for
+// a 128 x 256 x 16 MMA), so one commit per 4-MMA stage costs ~30% of the MMA
+// rate; a commit per two stages halves that but also halves the refill units
+// of the ring, which costs more than it saves when K is long (the operands
+// then stream from HBM for many k-blocks per tile).
+template <int BN, int STAGES, bool kSwap, int CG>
 __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
     using S = Shape<BN, kSwap>;
     constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
+    static_assert(STAGES % CG == 0, "stage groups");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
@@ -97,7 +104,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                 const CUtensorMap* bmap = &P.maps[pr.b_map[sg]];
                 const int kb_n = pr.kdim[sg] / kBK;
                 for (int kb = 0; kb < kb_n; ++kb) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, P.spin, err)) {
+                    // a group of CG stages is released by one commit: wait for it at the group's first stage
+                    if (stage % CG == 0 && !mbar_wait_bounded(&empty[stage / CG], phase ^ 1u, P.spin, err)) {
                         ok = false;
                         break;
                     }
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                         umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
                                   (kb > kb0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(&empty[stage]);
+                    if (stage % CG == CG - 1) umma_commit(&empty[stage / CG]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -514,16 +522,16 @@ constexpr size_t smem_bytes() {
     return 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 512;
 }
 
-template <int BN, int STAGES, bool kSwap>
+template <int BN, int STAGES, bool kSwap, int CG = 1>
 cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
     using S = Shape<BN, kSwap>;
     constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
     static_assert(smem <= 232448, "shared memory");
     static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 512, "barrier area");
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    k_gemm_tc<BN, STAGES, kSwap><<<grid, S::kThreads, smem, s>>>(P);
+    k_gemm_tc<BN, STAGES, kSwap, CG><<<grid, S::kThreads, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -566,6 +574,12 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
         if (tiles < grid) grid = (int)tiles;
         if (grid < 1) return cudaSuccess;
     }
+    // stage pairs per commit for short tiles (at most 32 k-blocks of K: the expert up GEMM at
+    // L = 2048, 4-5% faster); long-K tiles keep one commit per stage (8-10% slower with pairs)
+    bool short_k = true;
+    for (int i = 0; i < nprob; ++i)
+        short_k = short_k && probs[i].kdim[0] / kBK + (probs[i].nseg > 1 ? probs[i].kdim[1] / kBK : 0) <= 32;
+    if (short_k && bn == 256) return launch_impl<256, 4, false, 2>(P, grid, s);
     switch (bn) {
         case 256: return launch_impl<256, 4, false>(P, grid, s);
         case 128: return launch_impl<128, 6, false>(P, grid, s);
