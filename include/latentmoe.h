@@ -266,7 +266,10 @@ typedef enum {
                                     every routed expert of a token reads). Valid 0 .. 1e8. */
     LMOE_OPT_ACT_RECHECK_TAU = 5 /* threshold tau of the exact re-rounding of the relu2
                                     activations (expert and shared-expert up projections), in
-                                    1e-3 units (default 2000 = 2.0; 0 disables). bf16 mode,
+                                    1e-3 units (default 2000 = 2.0; 0 disables; values from 1
+                                    to 499 are refused: below tau = 0.5 the list, sized at
+                                    create, could not hold every activation the test can list,
+                                    whatever the inputs). bf16 mode,
                                     bf16 experts: an activation a = max(h, 0)^2 with h > tau whose
                                     fp32 value lies within the fp32 accumulation error of h
                                     (1.6e-6 + 0.9e-6 h, carried through the square) of a bf16
@@ -287,9 +290,9 @@ typedef struct {
     int z_rechecked;        /* z elements listed and re-rounded exactly (LMOE_OPT_Z_RECHECK_DELTA);
                                the list has room for all T*L elements                    */
     int ae_rechecked;       /* expert activations listed for exact re-rounding
-                               (LMOE_OPT_ACT_RECHECK_TAU); the list holds max(T*Is,
-                               T*top_k*expert_inter)/256 + 64 entries, and elements past
-                               it keep their fp32-decided rounding                      */
+                               (LMOE_OPT_ACT_RECHECK_TAU); the list has room for every
+                               activation the test can list at any accepted tau (about
+                               0.5% of max(T*Is, T*top_k*expert_inter))                 */
     int as_rechecked;       /* shared-expert activations listed, same list room          */
 } lmoe_stats;
 /* Reads the statistics of the last call that used ws (synchronises the device;

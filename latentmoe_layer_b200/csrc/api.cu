@@ -126,8 +126,9 @@ bool plan_of(const lmoe_config& c, int T, Plan& p) {
     // is large enough (top_k * I >= 4 L), else it has its own
     p.zlist = (A * I * act >= (size_t)T * L * 8) ? p.aperm : take((size_t)T * L * 8);
     // activation re-rounding list (the shared expert's, then the experts': one at a time), room
-    // for 1/256 of the larger activation set, far above the ~1e-4 that the margins list
-    p.alist_cap = (int)std::min<size_t>(std::max((size_t)T * Is, A * I) / 256 + 64, 0x7FFFFFFF);
+    // for every activation the flag test can list at any accepted tau (~0.5% of the larger set;
+    // ~0.02% is listed at the default tau on the synthetic workloads)
+    p.alist_cap = (int)std::min<size_t>(act_list_room(std::max((size_t)T * Is, A * I)), 0x7FFFFFFF);
     p.alist = take((size_t)p.alist_cap * 8);
     p.zrowtab = take((size_t)T * ((L + 2047) / 2048) * 16);  // one {row, first, entries} per 2048-column segment
     p.total = off;
@@ -318,8 +319,7 @@ void set_act_recheck(const Ctx& c, GemmProblem& pr, int* count) {
     const float tau2 = (float)(tau * tau);
     memcpy(&pr.rr_tau2_bits, &tau2, 4);
     // margin of a = h^2 over an fp32 ulp of a (>= a 2^-24), at its largest (a = tau^2)
-    pr.rr_ulps = (uint32_t)ceil(16777216.0 * (c0 / (tau * tau) + c0 + 2.0 * c1));
-    if (pr.rr_ulps > 0x4000u) pr.rr_ulps = 0x4000u;
+    pr.rr_ulps = act_margin_ulps(tau, c0, c1);
 }
 
 GemmProblem make_problem(int grouped, int m_rows, int n, int epi, void* out, long long ldo) {
@@ -915,7 +915,8 @@ lmoe_status latentmoe_set_option(lmoe_handle* h, lmoe_option opt, long long v) {
             h->spin_limit = (unsigned)v;
             return LMOE_OK;
         case LMOE_OPT_ACT_RECHECK_TAU:
-            if (v < 0 || v > 1000000) return LMOE_ERR_INVALID_ARG;
+            // 0 disables; below kActTauMin the list could not hold every flagged activation
+            if (v < 0 || v > 1000000 || (v > 0 && v * 1e-3 < kActTauMin)) return LMOE_ERR_INVALID_ARG;
             h->act_tau = (float)(v * 1e-3);
             return LMOE_OK;
     }

@@ -425,14 +425,15 @@ __global__ void __launch_bounds__(PairShape::kThreads, 1) k_gemm_tc_pair(const _
         for (int t = pair; t < ntiles && ok; t += npairs) {
             const TileInfo ti = pair_decode(P, t, rank);
             const int kb_total = tile_kblocks(P.prob[ti.p]);
-            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += CK) {
+            const int ck = P.prob[ti.p].chunk_kb ? P.prob[ti.p].chunk_kb : CK;
+            for (int kb0 = 0; kb0 < kb_total && ok; kb0 += ck) {
                 if (!mbar_wait_bounded(&cempty[buf], bphase ^ 1u, P.spin, err)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * BN);
-                const int kb1 = min(kb_total, kb0 + CK);
+                const int kb1 = min(kb_total, kb0 + ck);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
                         ok = false;
@@ -474,10 +475,11 @@ __global__ void __launch_bounds__(PairShape::kThreads, 1) k_gemm_tc_pair(const _
             const TileInfo ti = pair_decode(P, t, rank);
             const GemmProblem& pr = P.prob[ti.p];
             const int kb_total = tile_kblocks(pr);
+            const int ck = pr.chunk_kb ? pr.chunk_kb : CK;
             float acc[CW];
 #pragma unroll
             for (int i = 0; i < CW; ++i) acc[i] = 0.f;
-            for (int kb0 = 0; kb0 < kb_total; kb0 += CK) {
+            for (int kb0 = 0; kb0 < kb_total; kb0 += ck) {
                 if (!mbar_wait_bounded(&cfull[buf], bphase, P.spin, err)) {
                     ok = false;
                     break;

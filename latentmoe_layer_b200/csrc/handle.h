@@ -20,7 +20,7 @@ struct lmoe_handle {
     // (K = H = 8192) runs in chunks of 4 (measured on fc1, the same x and K: 1.16e-6 + 0.45e-6 h,
     // so the margin is 1.4-2x), the expert up GEMM (K = L = 2048) has a quarter of the chunks
     float act_tau = 2.0f;
-    float act_c0 = 1.6e-6f, act_c1 = 0.9e-6f;
+    float act_c0 = (float)lmoe::kActC0, act_c1 = (float)lmoe::kActC1;
     unsigned spin_limit = 1u << 24;
     int num_sms = 148;
     int launches = 0;                  // kernels launched by the last call

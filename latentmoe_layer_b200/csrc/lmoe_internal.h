@@ -101,6 +101,25 @@ struct GemmProblem {
     uint32_t rr_tau2_bits, rr_ulps;
 };
 
+// Accumulation-error margin c0 + c1 h of a relu2 pre-activation h, and the
+// smallest threshold the exact re-rounding of the activations accepts (below it
+// the margin, over a's fp32 ulp, grows as 1/tau^2 and the list would have to
+// be much larger).
+constexpr double kActC0 = 1.6e-6, kActC1 = 0.9e-6, kActTauMin = 0.5;
+// rr_flag's margin in fp32 ulps of a = h^2 at its largest relative size (a = tau^2).
+inline uint32_t act_margin_ulps(double tau, double c0, double c1) {
+    const double u = 16777216.0 * (c0 / (tau * tau) + c0 + 2.0 * c1);
+    return u >= 16384.0 ? 0x4000u : (uint32_t)u + 1u;
+}
+// List room that holds every activation rr_flag can list out of n, for any
+// tau >= kActTauMin: a listed value has its low 16 bits in a window of
+// 2 * ulps of the 65536 patterns around 0x8000, and the window's share is
+// largest at the smallest tau.
+inline size_t act_list_room(size_t n) {
+    const size_t w = 2u * act_margin_ulps(kActTauMin, kActC0, kActC1);
+    return n / 65536 * w + ((n % 65536) * w + 65535) / 65536 + 64;
+}
+
 // Whether a = max(h, 0)^2, computed in fp32, is above tau^2 and within `ulps`
 // fp32 ulps of a bf16 rounding midpoint. For a positive fp32 value the bf16
 // values are the patterns with zero low 16 bits and the only midpoint between

@@ -172,6 +172,10 @@ def test_call_errors_leave_outputs_untouched(lib):
     assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 100000001) == lm.LMOE_ERR_INVALID_ARG
     assert lm.latentmoe_set_option(layer.h, lm.OPT_Z_RECHECK_DELTA, 0) == lm.LMOE_OK
     assert lm.latentmoe_set_option(layer.h, lm.OPT_ACT_RECHECK_TAU, -1) == lm.LMOE_ERR_INVALID_ARG
+    # below tau = 0.5 the re-rounding list could not hold every activation the flag test lists
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_ACT_RECHECK_TAU, 499) == lm.LMOE_ERR_INVALID_ARG
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_ACT_RECHECK_TAU, 500) == lm.LMOE_OK
+    assert lm.latentmoe_set_option(layer.h, lm.OPT_ACT_RECHECK_TAU, 0) == lm.LMOE_OK
     assert lm.latentmoe_set_option(layer.h, 6, 0) == lm.LMOE_ERR_INVALID_ARG
 
 
