@@ -341,10 +341,12 @@ lmoe_status latentmoe_route_noalloc(lmoe_handle* h, const void* x, int T, int32_
 
 /* Stage markers for timing inside a real call: when set (n >= 8), the next
  * latentmoe_forward calls record events[i] (cudaEvent_t) on their stream at
- * stage boundary i: 0 start, 1 routing done (router GEMM, selection, fp64
- * re-check, permutation), 2 input GEMM (fc1 + shared up) done, 3 gather done,
- * 4 expert up GEMM done, 5 expert down GEMM done, 6 combine done, 7 output
- * GEMM done. NULL turns it off. The events are borrowed and must exist (a
+ * stage boundary i: 0 start, 1 routing head done (the statistics reset, and
+ * the router GEMM when it cannot be the first problem of the input GEMM
+ * launch), 2 input stage done (the input GEMM; selection, fp64 re-check and
+ * permutation on the second stream; the exact re-roundings of z and a_s),
+ * 3 gather done, 4 expert up GEMM done, 5 expert down GEMM done, 6 combine
+ * done, 7 output GEMM done. NULL turns it off. The events are borrowed and must exist (a
  * NULL event among the first 8 returns LMOE_ERR_INVALID_ARG); a record that
  * fails is skipped and does not fail the call it times. */
 lmoe_status latentmoe_set_profile_events(lmoe_handle* h, void* const* events, int n);
