@@ -42,16 +42,29 @@ namespace lmoe {
 namespace {
 
 // CG: shared-memory stages released per MMA commit. A tcgen05.commit holds the
-// tensor pipe for about an MMA's latency (~230 cycles measured, against 130 for
-// a 128 x 256 x 16 MMA), so one commit per 4-MMA stage costs ~30% of the MMA
-// rate; a commit per two stages halves that but also halves the refill units
-// of the ring, which costs more than it saves when K is long (the operands
-// then stream from HBM for many k-blocks per tile).
-template <int BN, int STAGES, bool kSwap, int CG>
-__global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+// issuing thread's MMAs for about an MMA's latency (~230 cycles measured,
+// against 130 for a 128 x 256 x 16 MMA), so one commit per 4-MMA stage costs
+// ~30% of the MMA rate; a commit per two stages halves that but also halves the
+// refill units of the ring, which costs more than it saves when K is long (the
+// operands then stream from HBM for many k-blocks per tile). A second issuing
+// thread hides much of it too (two threads committing every 4 MMAs: 156 cycles
+// per MMA against 189.6 for one).
+//
+// NIS: MMA-issuing threads. With two (lane 0 of warp 1 and of an extra warp
+// after the epilogue warps), issuer i takes the k-blocks of parity i into its
+// own TMEM accumulator (buffer i), so each commits after every stage it used
+// while the other's MMAs keep the tensor pipe busy. A chunk then spans 2 * ck
+// k-blocks, ck in each accumulator, and the epilogue adds buffer 0, then
+// buffer 1, into its registers: the partial sums have the single-issuer
+// chunk's length. Needs an even k-block count in every tile (the parity then
+// carries across tiles) and an even stage count (a stage keeps its issuer).
+template <int BN, int STAGES, bool kSwap, int CG, int NIS>
+__global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads + (NIS - 1) * 32, 1)
+    k_gemm_tc(const __grid_constant__ TcParams P) {
     using S = Shape<BN, kSwap>;
     constexpr int NB = S::kBufs, CK = S::kChunkKB, CW = S::kColsPerThread;
     static_assert(STAGES % CG == 0, "stage groups");
+    static_assert(NIS == 1 || (NIS == 2 && NB == 2 && CG == 1 && STAGES % 2 == 0 && !kSwap), "two issuers");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((base_u32 + 1023u) & ~1023u) - base_u32);
@@ -62,10 +75,11 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
     uint64_t* empty = full + STAGES;
     uint64_t* cfull = empty + STAGES;   // chunk accumulator ready (MMA -> epilogue)
     uint64_t* cempty = cfull + NB;      // chunk accumulator drained (epilogue -> MMA)
-    uint64_t* done = cempty + NB;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* done = cempty + NB;       // one per issuer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + NIS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kIssuer2Warp = S::kThreads / 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -75,7 +89,7 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
             mbar_init(&cfull[b], 1);
             mbar_init(&cempty[b], S::kEpiWarps);
         }
-        mbar_init(done, 1);
+        for (int i = 0; i < NIS; ++i) mbar_init(&done[i], 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0)
@@ -129,17 +143,18 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
         // every load this thread issued has landed before the CTA can exit
         for (int s = 0; s < STAGES; ++s)
             if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, 1u << 26, err);
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------ MMA issuer
+    } else if (lane == 0 && (warp == 1 || (NIS == 2 && warp == kIssuer2Warp))) {
+        // ------------------------------------------------ MMA issuer(s)
         constexpr uint32_t idesc_full = idesc_bf16_f32(128, BN);
         constexpr uint32_t idesc_half = idesc_bf16_f32(64, BN);
-        int stage = 0, buf = 0;
+        const int ii = warp == 1 ? 0 : 1;  // this issuer's k-block parity (NIS == 2)
+        int stage = NIS == 2 ? ii : 0, buf = NIS == 2 ? ii : 0;
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN, kSwap>(P, t);
             const int kb_total = tile_kblocks(P.prob[ti.p]);
-            const int ck = P.prob[ti.p].chunk_kb ? P.prob[ti.p].chunk_kb : CK;
+            const int ck = (P.prob[ti.p].chunk_kb ? P.prob[ti.p].chunk_kb : CK) * NIS;
             // M = 64 puts D rows 16q..16q+15 in TMEM lanes 32q..32q+15 (q = lane quarter)
             const uint32_t idesc = ti.half ? idesc_half : idesc_full;
             for (int kb0 = 0; kb0 < kb_total && ok; kb0 += ck) {
@@ -151,7 +166,8 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * BN);
                 const int kb1 = min(kb_total, kb0 + ck);
-                for (int kb = kb0; kb < kb1; ++kb) {
+                const int kbs = kb0 + (NIS == 2 ? ii : 0);
+                for (int kb = kbs; kb < kb1; kb += NIS) {
                     if (!mbar_wait_bounded(&full[stage], phase, P.spin, err)) {
                         ok = false;
                         break;
@@ -163,26 +179,29 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // +32 bytes per K step of 16 bf16 inside the 128-byte swizzled row
                         umma_bf16(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
-                                  (kb > kb0 || kk > 0) ? 1u : 0u);
+                                  (kb > kbs || kk > 0) ? 1u : 0u);
                     }
                     if (stage % CG == CG - 1) umma_commit(&empty[stage / CG]);
-                    if (++stage == STAGES) {
-                        stage = 0;
+                    stage += NIS;
+                    if (stage >= STAGES) {
+                        stage -= STAGES;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
                 umma_commit(&cfull[buf]);
-                if (++buf == NB) {
+                if (NIS == 2) {
+                    bphase ^= 1u;  // this issuer's one buffer, once per chunk
+                } else if (++buf == NB) {
                     buf = 0;
                     bphase ^= 1u;
                 }
             }
         }
         // all MMAs issued by this thread have completed before TMEM is freed
-        umma_commit(done);
-        mbar_wait_bounded(done, 0, 1u << 26, err);
-    } else if (warp >= 2) {
+        umma_commit(&done[ii]);
+        mbar_wait_bounded(&done[ii], 0, 1u << 26, err);
+    } else if (warp >= 2 && warp < 2 + S::kEpiWarps) {
         // ------------------------------------------------ epilogue
         const int ew = warp - 2;
         const int q = warp & 3;                // TMEM lane quarter this warp may access
@@ -205,7 +224,9 @@ __global__ void __launch_bounds__(Shape<BN, kSwap>::kThreads, 1) k_gemm_tc(const
 #pragma unroll
             for (int i = 0; i < CW; ++i) acc[i] = 0.f;
 #endif
-            for (int kb0 = 0; kb0 < kb_total; kb0 += ck) {
+            // NIS == 2: chunks of 2 ck k-blocks, one partial in each buffer, added in buffer order
+            const int nparts = NIS * ((kb_total + ck * NIS - 1) / (ck * NIS));
+            for (int part = 0; part < nparts; ++part) {
                 if (!mbar_wait_bounded(&cfull[buf], bphase, P.spin, err)) {
                     ok = false;
                     break;
@@ -524,16 +545,16 @@ constexpr size_t smem_bytes() {
     return 1024 + (size_t)STAGES * S::kStageBytes + (size_t)S::kEpiWarps * S::kStageOutBytes + 512;
 }
 
-template <int BN, int STAGES, bool kSwap, int CG = 1>
+template <int BN, int STAGES, bool kSwap, int CG = 1, int NIS = 1>
 cudaError_t launch_impl(const TcParams& P, int grid, cudaStream_t s) {
     using S = Shape<BN, kSwap>;
     constexpr size_t smem = smem_bytes<BN, STAGES, kSwap>();
     static_assert(smem <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * S::kBufs + 1) * 8 + 4 <= 512, "barrier area");
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    static_assert((2 * STAGES + 2 * S::kBufs + NIS) * 8 + 4 <= 512, "barrier area");
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, kSwap, CG, NIS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_gemm_tc<BN, STAGES, kSwap, CG><<<grid, S::kThreads, smem, s>>>(P);
+    k_gemm_tc<BN, STAGES, kSwap, CG, NIS><<<grid, S::kThreads + (NIS - 1) * 32, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -576,12 +597,20 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
         if (tiles < grid) grid = (int)tiles;
         if (grid < 1) return cudaSuccess;
     }
-    // stage pairs per commit for short tiles (at most 32 k-blocks of K: the expert up GEMM at
-    // L = 2048, 4-5% faster); long-K tiles keep one commit per stage (8-10% slower with pairs)
-    bool short_k = true;
-    for (int i = 0; i < nprob; ++i)
-        short_k = short_k && probs[i].kdim[0] / kBK + (probs[i].nseg > 1 ? probs[i].kdim[1] / kBK : 0) <= 32;
-    if (short_k && bn == 256) return launch_impl<256, 4, false, 2>(P, grid, s);
+    bool short_k = true, even_k = true;
+    for (int i = 0; i < nprob; ++i) {
+        const int kbt = probs[i].kdim[0] / kBK + (probs[i].nseg > 1 ? probs[i].kdim[1] / kBK : 0);
+        short_k = short_k && kbt <= 32;
+        even_k = even_k && kbt % 2 == 0;
+    }
+    // short tiles (at most 32 k-blocks: the expert up GEMM at L = 2048): two MMA issuers, or one
+    // commit per two stages when a tile's k-block count is odd. Long-K tiles keep one issuer
+    // with a commit per stage: both other forms cost them 8-10% (each issuer's chunk drains are
+    // no longer hidden behind a second buffer; stage pairs halve the ring's refill units).
+    if (short_k && bn == 256) {
+        if (even_k) return launch_impl<256, 4, false, 1, 2>(P, grid, s);
+        return launch_impl<256, 4, false, 2>(P, grid, s);
+    }
     switch (bn) {
         case 256: return launch_impl<256, 4, false>(P, grid, s);
         case 128: return launch_impl<128, 6, false>(P, grid, s);

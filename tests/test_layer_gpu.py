@@ -67,12 +67,17 @@ def test_pair_widths_bf16(path):
     run_and_compare(PAIRW, mode=0, path=path)
 
 
+# every GEMM's K above 32 k-blocks of 64 (single-CTA tiles then have one MMA issuer), widths multiples
+# of 256 (pair tiles)
+PAIRL = LayerShape("pair_long_k", T=600, H=2304, L=2304, E=16, k=4, G=4, Gk=2, I=2304, Is=2304)
+
+
 def test_pair_tiles_give_the_single_cta_result_bit_for_bit():
     """A 2-SM pair tile (M = 256 over two CTAs) accumulates each CTA's 128 rows in the same K order and
     TMEM chunks (per problem: fc1 and the shared up projection in chunks of 4 k-blocks) as a single-CTA
-    tile, so the whole layer output is the same bits on both prefill paths."""
+    tile with one MMA issuer, so the whole layer output is the same bits on both prefill paths."""
     import torch
-    shape = PAIRW
+    shape = PAIRL
     layer, dev = H.device_layer(shape)
     ys = []
     for path in (GEMM_PREFILL, GEMM_PREFILL_PAIR):
