@@ -316,11 +316,11 @@ def measure(shape, steps, warmup, world, rank, local, dist, torch, nvfp4=False):
 
 
 # DRAM bytes per assignment of the expert up GEMM, from an ncu capture of this
-# kernel on the probe_e64 workload (1.981 GB for 45 056 assignments; the same
+# kernel on the probe_e64 workload (1.978 GB for 45 056 assignments; the same
 # tile shapes and rows per expert as ultra_prefill). Traffic grows with the
 # assignments (rows) and, at ~704 rows per expert, with the experts in the same
 # ratio. Reset to None when that kernel changes.
-UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT = (1.529e9 + 0.452e9) / 45056
+UP_GEMM_DRAM_BYTES_PER_ASSIGNMENT = (1.529e9 + 0.449e9) / 45056
 
 
 def roofline_for(shape, res, peaks, peak_src, prefill: bool, nvfp4=False):
