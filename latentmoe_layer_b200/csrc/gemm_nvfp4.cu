@@ -257,8 +257,9 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS, NB, NI, SL>:
                 const int kb1 = min(kb_n, kb0 + CK);
                 for (int kb = kb0; kb < kb1; kb += KB, ++c) {
                     const int s = (int)(c % STAGES);
-                    if (!mbar_wait_bounded(&deq[s], (c / STAGES) & 1u, spin, err) ||
-                        !mbar_wait_bounded(&full[s], (c / STAGES) & 1u, spin, err)) {
+                    // deq[s] completes only after every dequantisation warp has seen full[s]
+                    // complete, so the stage's copies (the token tiles included) have landed
+                    if (!mbar_wait_bounded(&deq[s], (c / STAGES) & 1u, spin, err)) {
                         ok = false;
                         break;
                     }
@@ -310,11 +311,24 @@ __global__ void __launch_bounds__(Fp4TmShape<BN, STAGES, KB, G, AS, NB, NI, SL>:
                     break;
                 }
                 const uint8_t* st = smem + s * F::kStageBytes;
+                // every shared-memory load of this warp's k-blocks of the stage first (codes and
+                // scale bytes), then the conversions and TMEM stores
+                constexpr int NJ = KB / G;
+                uint4 cw[NJ][2];
+                uint32_t sbw[NJ];
 #pragma unroll
-                for (int j = grp; j < KB; j += G) {
+                for (int u = 0; u < NJ; ++u) {
+                    const int j = grp + u * G;
                     const uint8_t* codes = st + F::kOffCodes + j * 4096 + row * 32;
-                    const uint4 c0 = ld_shared_v4(codes), c1 = ld_shared_v4(codes + 16);
-                    const uint32_t sb = ld_shared_u32(st + F::kOffSf + j * 512 + row * 4);
+                    cw[u][0] = ld_shared_v4(codes);
+                    cw[u][1] = ld_shared_v4(codes + 16);
+                    sbw[u] = ld_shared_u32(st + F::kOffSf + j * 512 + row * 4);
+                }
+#pragma unroll
+                for (int u = 0; u < NJ; ++u) {
+                    const int j = grp + u * G;
+                    const uint4 c0 = cw[u][0], c1 = cw[u][1];
+                    const uint32_t sb = sbw[u];
                     uint4 os[8];
                     if constexpr (SL) {
                         const uint4* tl = reinterpret_cast<const uint4*>(scale_lut);
