@@ -293,7 +293,8 @@ cudaError_t run_gemm_nvfp4(Ctx& c, GemmProblem* pr, const Operand& act) {
 
 // TMEM accumulation chunks (k-blocks of 64) per GEMM: a chunk bounds the size of
 // the partial sums the tensor core accumulates, which matters where the output
-// is rounded to bf16; fp32 outputs (expert down, output GEMM) take K whole.
+// is rounded to bf16 (0: the engine's default of 8 k-blocks, also taken by the
+// fp32 outputs of the expert down and output GEMMs).
 #ifndef LMOE_CHUNK_UP
 #define LMOE_CHUNK_UP 0      // expert up (a_e, re-rounded): the engine's default
 #endif

@@ -90,6 +90,18 @@ def test_pair_tiles_give_the_single_cta_result_bit_for_bit():
     assert torch.equal(ys[0], ys[1])
 
 
+# odd k-block counts on 256-wide tiles: the expert up GEMM (K = L = 320, five k-blocks; N = I = 512)
+# runs the single-issuer form with one commit per two stages (the two-issuer form needs an even count),
+# the shared up projection (K = H = 576, nine; N = Is = 768) likewise inside the input launch
+ODDK = LayerShape("odd_kblocks", T=300, H=576, L=320, E=32, k=4, G=4, Gk=2, I=512, Is=768)
+
+
+def test_odd_kblock_tiles():
+    (ma, rf), layer = run_and_compare(ODDK, mode=0, path=GEMM_PREFILL)
+    assert layer.stats().device_error == 0
+    print("odd_kblocks max_abs=%.3g rel_fro=%.3g" % (ma, rf))
+
+
 # T = 40 at decode sizes: the input GEMM (router merged, (128 + 2048 + 8192) / 128 = 81 weight tiles)
 # runs one wave of 64-token tiles, each holding 40 valid tokens, instead of two waves of 32-token tiles
 DEC64 = LayerShape("decode_64_tiles", T=40, H=1024, L=2048, E=128, k=4, G=4, Gk=2, I=512, Is=8192)
