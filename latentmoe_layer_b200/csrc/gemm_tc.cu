@@ -605,8 +605,9 @@ cudaError_t launch_gemm_tc(const CUtensorMap* maps, int nmaps, const GemmProblem
     }
     // short tiles (at most 32 k-blocks: the expert up GEMM at L = 2048): two MMA issuers, or one
     // commit per two stages when a tile's k-block count is odd. Long-K tiles keep one issuer
-    // with a commit per stage: both other forms cost them 8-10% (each issuer's chunk drains are
-    // no longer hidden behind a second buffer; stage pairs halve the ring's refill units).
+    // with a commit per stage: both other forms cost them 3-10% (with two issuers interleaved in
+    // the tensor pipe each stage is released later; stage pairs halve the ring's refill units),
+    // which matters where the operands stream from HBM.
     if (short_k && bn == 256) {
         if (even_k) return launch_impl<256, 4, false, 1, 2>(P, grid, s);
         return launch_impl<256, 4, false, 2>(P, grid, s);
