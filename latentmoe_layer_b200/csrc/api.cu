@@ -192,15 +192,15 @@ int pick_bn(const int* ns, int cnt) {
 }
 
 // Tokens per tile of a swap-AB (decode) launch: 64 where every problem is dense
-// with at most 64 rows and 64-token tiles take fewer waves over the SMs than
-// 32-token ones (each wave streams the same weight tiles; more tiles in a wave
-// keep more SMs streaming), else kDecodeTN.
+// and 64-token tiles take fewer waves over the SMs than 32-token ones (each
+// token tile streams the same weight tiles again; at equal waves more tiles in a
+// wave keep more SMs streaming), else kDecodeTN.
 int decode_bn(const GemmProblem* probs, int nprob, int sms) {
     long long t32 = 0, t64 = 0;
     for (int i = 0; i < nprob; ++i) {
-        if (probs[i].grouped || probs[i].m_rows > 64) return kDecodeTN;
+        if (probs[i].grouped) return kDecodeTN;
         t32 += (long long)((probs[i].m_rows + kDecodeTN - 1) / kDecodeTN) * (probs[i].n / 128);
-        t64 += probs[i].n / 128;
+        t64 += (long long)((probs[i].m_rows + 63) / 64) * (probs[i].n / 128);
     }
     return (t64 + sms - 1) / sms < (t32 + sms - 1) / sms ? 64 : kDecodeTN;
 }
