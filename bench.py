@@ -345,16 +345,12 @@ def roofline_for(shape, res, peaks, peak_src, prefill: bool, nvfp4=False):
             "algorithmic_per_launch": byts, "launch_ms": round(kms, 4)}
 
 
-L2_BYTES = 126e6
-
-
 def target_of(shape, summary, prefill):
     """The layer-level target the throughput is held to: >= 60% of the bf16 tensor
     peak (burst) at large token counts, >= 70% of HBM bandwidth over the touched
     weights at decode sizes. A layer whose weights fit in L2 is latency-bound:
     reported, with no target."""
-    import latentmoe_layer_b200.accounting as acc
-    if acc.min_bytes_per_call(shape, shape.E) < L2_BYTES:
+    if weight_bytes_of(shape) < L2_BYTES:
         return {"metric": None, "value": None, "target": None, "met": None,
                 "note": "latency-bound (the weights fit in L2): reported only"}
     key, goal = ("layer_frac_of_burst_bf16", 0.60) if prefill else ("layer_frac_of_hbm", 0.70)

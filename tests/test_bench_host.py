@@ -49,6 +49,20 @@ def test_l2_flush_only_for_weights_that_fit_in_l2():
     assert abs(bench.weight_bytes_of(ULTRA_PREFILL) / 1e9 - 21.886) < 0.01
 
 
+def test_no_target_for_a_layer_whose_weights_fit_in_l2():
+    """A latency-bound layer (its weights fit in L2) is reported with no target; the others are held to
+    60% of the burst bf16 peak at prefill sizes and 70% of HBM at decode sizes."""
+    sys.path.insert(0, ROOT)
+    import bench
+    summary = {"layer_frac_of_burst_bf16": 0.7, "layer_frac_of_hbm": 0.5}
+    t = bench.target_of(TINY, summary, prefill=False)
+    assert t["target"] is None and t["met"] is None and "latency" in t["note"]
+    t = bench.target_of(ULTRA_PREFILL, summary, prefill=True)
+    assert t == {"metric": "layer_frac_of_burst_bf16", "value": 0.7, "target": 0.6, "met": True}
+    t = bench.target_of(NANO_DECODE, summary, prefill=False)
+    assert t == {"metric": "layer_frac_of_hbm", "value": 0.5, "target": 0.7, "met": False}
+
+
 def test_one_core_baseline_restores_the_thread_count(built_oracle):
     import ctypes
     import torch
